@@ -1,0 +1,558 @@
+#!/usr/bin/env python
+"""Benchmark of decode-step combined sparse attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one decode step of one full-attention layer on the 64k workload:
+B=4 sequences of 65536 tokens (+1 per step), 32 query / 4 kv heads, head_dim
+128, 16-token pages, prefix 128, window 1024, budget 128 pages, 64 planted
+needles per sequence.  Each step appends the new token (kv_append, which also
+updates the page bounds) and runs the sparse decode (score, select, attend,
+merge).  The 256k workload (B=4, 262144 tokens, window 4096, budget 256) and
+the dense flash-decode kernel over the same caches are measured after the
+timed region and reported under "also".
+
+Rank 0 prints one JSON line.  With N > 1 (torchrun), every rank runs its own
+replica (weak scaling); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse decode-attn µs/step/layer & HBM GB/s at 64k/256k, B=4; speedup vs dense"
+UNIT = "us/step/layer"
+FLUSH_BYTES = 256 << 20  # > 2x the 126 MB L2
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=256)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-also", action="store_true", help="skip the 256k/dense measurements")
+    ap.add_argument("--reps", type=int, default=20, help="repetitions of each extra measurement")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- helpers
+
+def rank_info():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def page_ranges(L, prefix, window):
+    """Page ranges of the method (pages [0,np) prefix, [np,ws) candidates,
+    [ws,n) window) -- used here only to count algorithmic bytes."""
+    n = -(-L // 16) if L > 0 else 0
+    np_ = min(-(-prefix // 16), n)
+    ws = n if window <= 0 else max(L - window, 0) // 16
+    ws = min(max(ws, np_), n)
+    return n, np_, ws
+
+
+def algorithmic_bytes(lens, hq, hkv, D, prefix, window, budget, dense=False):
+    """Bytes the step must move: metadata of candidate pages (4*D per page
+    and kv head), K and V of attended tokens (4*D per token and kv head), q
+    (bf16) and out (fp32).  Returns (total, meta, kv)."""
+    meta = kv = 0
+    for L in lens:
+        n, np_, ws = page_ranges(L, prefix, window)
+        if dense:
+            tokens = L
+        else:
+            nc = ws - np_
+            meta += nc * hkv * 4 * D
+            sel = min(budget, nc)
+            tokens = min(L, 16 * np_) + 16 * sel + max(0, L - 16 * ws)
+        kv += tokens * hkv * 4 * D
+    qo = len(lens) * hq * D * (2 + 4)
+    return meta + kv + qo, meta, kv
+
+
+class Clocks:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+    def __init__(self, index):
+        self.samples, self.reasons = [], 0
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report nothing rather than guess
+            self.err = str(e)
+        self.stop_flag = threading.Event()
+        self.t = None
+
+    def _run(self):
+        nv = self.nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(get_r(self.h))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.t:
+            self.stop_flag.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and bit != 0x1]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples), "reasons": names}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def ncu_traffic():
+    """Per-launch DRAM bytes from the committed ncu summary, keyed by kernel
+    and workload, valid only while the kernel source is unchanged."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.md")
+    out = {}
+    if not os.path.exists(path):
+        return out
+    csrc = os.path.join(ROOT, "sparse_long_context_max_b200", "csrc")
+    for line in open(path):
+        parts = [p.strip() for p in line.strip().strip("|").split("|")]
+        if len(parts) != 5 or not parts[2].isdigit():
+            continue
+        kernel, workload, nbytes, src, sha = parts
+        try:
+            cur = hashlib.sha1(open(os.path.join(csrc, src), "rb").read()).hexdigest()[:12]
+        except OSError:
+            continue
+        if cur == sha:
+            out[(kernel, workload)] = int(nbytes)
+    return out
+
+
+# ----------------------------------------------------------------- GPU arm
+
+class Workload:
+    """Device-resident inputs of one workload (single layer)."""
+
+    def __init__(self, name, extra_tokens=0):
+        import torch
+        import sparse_long_context_max_b200 as slc
+        import synth
+        self.wl = synth.WORKLOADS[name]
+        self.x = synth.make_inputs(self.wl, headroom_tokens=extra_tokens)
+        x = self.x
+        self.q = x.q.cuda()
+        self.k = x.k_cache.cuda()
+        self.v = x.v_cache.cuda()
+        self.bt = x.block_table.cuda()
+        self.sl = x.seq_lens.cuda()
+        self.cache = slc.PagedCache(self.k, self.v)
+        slc.build_page_meta(self.cache, self.bt, self.sl)
+        B, hq, D = x.q.shape
+        self.out = torch.empty((B, hq, D), dtype=torch.float32, device="cuda")
+        K = max(x.budget, 1)
+        self.sel = torch.empty((B, self.wl.hkv, K), dtype=torch.int32, device="cuda")
+        self.ws = torch.empty(slc.workspace_size(B, hq, self.wl.hkv, D, x.block_table.shape[1],
+                                                 x.budget), dtype=torch.uint8, device="cuda")
+        self.scores = torch.empty((B, self.wl.hkv, x.block_table.shape[1]),
+                                  dtype=torch.float32, device="cuda")
+
+
+def timed(fn, reps, flush, warm=3):
+    """Average device time (ms) of fn() over reps, L2 flushed before each."""
+    import torch
+    for _ in range(warm):
+        fn()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    torch.cuda.synchronize()
+    torch.cuda._sleep(5_000_000)  # let the host queue ahead of the device
+    for s, e in ev:
+        flush.zero_()
+        s.record()
+        fn()
+        e.record()
+    torch.cuda.synchronize()
+    return sum(s.elapsed_time(e) for s, e in ev) / reps
+
+
+def graph_of(fn):
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # warm (first-call set-up happens outside capture)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+    import sparse_long_context_max_b200 as slc
+    import synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    K, Wm = args.steps, args.warmup
+
+    # ---- primary workload: 64k decode loop with appends
+    W64 = Workload("decode64k", extra_tokens=K + Wm)
+    x, wl = W64.x, W64.wl
+    B, hq, hkv, D = wl.batch, wl.hq, wl.hkv, wl.head_dim
+    L0 = x.seq_lens.clone()
+    nsteps = K + Wm
+    qs, kns, vns = [], [], []
+    for t in range(nsteps):
+        q, kn, vn = synth.step_tokens(wl, 1 + t)
+        qs.append(q)
+        kns.append(kn)
+        vns.append(vn)
+    q_all = torch.stack(qs).cuda()
+    kn_all = torch.stack(kns).cuda()
+    vn_all = torch.stack(vns).cuda()
+    pos_all = torch.stack([L0 + t for t in range(nsteps)]).to(torch.int32).cuda()
+    len_all = (pos_all + 1).contiguous()
+    cur_q = torch.empty_like(q_all[0])
+    cur_kn = torch.empty_like(kn_all[0])
+    cur_vn = torch.empty_like(vn_all[0])
+    cur_pos = torch.empty_like(pos_all[0])
+    cur_len = torch.empty_like(len_all[0])
+
+    def step():
+        slc.kv_append(W64.cache, cur_kn, cur_vn, W64.bt, cur_pos)
+        slc.sparse_decode(cur_q, W64.cache, W64.bt, cur_len, x.prefix, x.window, x.budget,
+                          out=W64.out, workspace=W64.ws)
+
+    def stage(t):
+        cur_q.copy_(q_all[t])
+        cur_kn.copy_(kn_all[t])
+        cur_vn.copy_(vn_all[t])
+        cur_pos.copy_(pos_all[t])
+        cur_len.copy_(len_all[t])
+
+    stage(0)
+    g = graph_of(step)  # runs step 0 twice (append is idempotent for one token)
+    for t in range(1, Wm):
+        stage(t)
+        g.replay()
+    torch.cuda.synchronize()
+    assert slc.device_status() == 0
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = Clocks(local)
+    with clocks:
+        t_wall = time.perf_counter()
+        torch.cuda._sleep(20_000_000)
+        for i, (s, e) in enumerate(ev):
+            stage(Wm + i)
+            flush.zero_()
+            s.record()
+            g.replay()
+            e.record()
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        dist.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    assert slc.device_status() == 0
+    ms_per_step = total_ms / K
+    us_step = ms_per_step * 1e3
+    value = us_step / world  # time per step-layer over the whole job
+    lens_mid = [int(v) + Wm + K // 2 for v in L0]
+    step_bytes, meta_b, kv_b = algorithmic_bytes(lens_mid, hq, hkv, D, x.prefix, x.window,
+                                                 x.budget)
+    step_bytes += B * hkv * (2 * D * 2 + 2 * 2 * D * 2)  # append: k, v + meta read/write
+    peak, peak_kind = measured_peak()
+    traffic = ncu_traffic()
+
+    # ---- per-kernel device times on the 64k state (standalone entry points)
+    reps = args.reps
+    stage(Wm + K - 1)
+    sel64 = W64.sel[:, :, :x.budget]
+    kt = {}
+    kt["score_pages"] = timed(lambda: slc.score_pages(cur_q, W64.cache, W64.bt, cur_len, x.prefix,
+                                                       x.window, scores=W64.scores), reps, flush)
+    kt["select_pages"] = timed(lambda: slc.select_pages(W64.scores, cur_len, x.prefix, x.window,
+                                                         x.budget, selected=sel64), reps, flush)
+    kt["sparse_attend"] = timed(lambda: slc.sparse_attend(cur_q, W64.cache, W64.bt, cur_len,
+                                                          x.prefix, x.window, sel64, out=W64.out,
+                                                          workspace=W64.ws), reps, flush)
+    kt["kv_append"] = None  # measured inside the step only (its state changes)
+    _, meta64, kv64 = algorithmic_bytes([int(v) + Wm + K for v in L0], hq, hkv, D, x.prefix,
+                                        x.window, x.budget)
+    kbytes = {"score_pages": meta64 + B * hq * D * 2, "sparse_attend": kv64 + B * hq * D * 6}
+    dom = max(("score_pages", "sparse_attend"), key=lambda k: kt[k])
+    ach = kbytes[dom] / (kt[dom] * 1e-3) / 1e9
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(ach / peak, 4),
+                "traffic": traffic.get((dom, "decode64k")),
+                "algorithmic_bytes": kbytes[dom], "us_per_launch": round(kt[dom] * 1e3, 2),
+                "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind}
+
+    # ---- dense comparison on the same 64k cache
+    also = {}
+    if not args.no_also:
+        dense64 = timed(lambda: slc.dense_decode(cur_q, W64.cache, W64.bt, cur_len, out=W64.out,
+                                                 workspace=W64.ws), reps, flush)
+        sparse64 = timed(lambda: slc.sparse_decode(cur_q, W64.cache, W64.bt, cur_len, x.prefix,
+                                                   x.window, x.budget, out=W64.out,
+                                                   workspace=W64.ws), reps, flush)
+        db, _, _ = algorithmic_bytes([int(v) + Wm + K for v in L0], hq, hkv, D, 0, 0, 0, True)
+        also["decode64k"] = {
+            "sparse_us": round(sparse64 * 1e3, 2), "dense_us": round(dense64 * 1e3, 2),
+            "speedup_vs_dense": round(dense64 / sparse64, 2),
+            "dense_gbs": round(db / (dense64 * 1e-3) / 1e9, 1),
+            "kernel_us": {k: (round(v * 1e3, 2) if v else None) for k, v in kt.items()}}
+
+    # ---- e2e through the public API: host buffers, copies inside the timing
+    qh = torch.stack(qs).pin_memory()
+    knh = torch.stack(kns).pin_memory()
+    vnh = torch.stack(vns).pin_memory()
+    posh = torch.stack([L0 + t for t in range(nsteps)]).to(torch.int32).pin_memory()
+    lenh = (posh + 1).pin_memory()
+    outh = torch.empty((B, hq, D), dtype=torch.float32).pin_memory()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+    torch.cuda.synchronize()
+    for i, (s, e) in enumerate(e2e_ev):
+        t = Wm + i
+        flush.zero_()
+        s.record()
+        cur_q.copy_(qh[t], non_blocking=True)
+        cur_kn.copy_(knh[t], non_blocking=True)
+        cur_vn.copy_(vnh[t], non_blocking=True)
+        cur_pos.copy_(posh[t], non_blocking=True)
+        cur_len.copy_(lenh[t], non_blocking=True)
+        slc.kv_append(W64.cache, cur_kn, cur_vn, W64.bt, cur_pos)
+        slc.sparse_decode(cur_q, W64.cache, W64.bt, cur_len, x.prefix, x.window, x.budget,
+                          out=W64.out, workspace=W64.ws)
+        outh.copy_(W64.out, non_blocking=True)
+        e.record()
+    torch.cuda.synchronize()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in e2e_ev)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    h2d = (qh[0].numel() * 2 + knh[0].numel() * 2 + vnh[0].numel() * 2 + posh[0].numel() * 4
+           + lenh[0].numel() * 4)
+    e2e = {"value": round(e2e_ms * 1e3 / K / world, 3), "unit": UNIT,
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(outh.numel() * 4),
+           "path": "binding calls kv_append + sparse_decode (eager), pinned host copies"}
+
+    # ---- 256k workload: sparse vs dense, per-kernel roofline
+    if not args.no_also:
+        del qs, kns, vns
+        W256 = Workload("decode256k")
+        y = W256.x
+        b256 = algorithmic_bytes(y.seq_lens.tolist(), y.wl.hq, y.wl.hkv, y.wl.head_dim,
+                                 y.prefix, y.window, y.budget)
+        sp = timed(lambda: slc.sparse_decode(W256.q, W256.cache, W256.bt, W256.sl, y.prefix,
+                                             y.window, y.budget, out=W256.out,
+                                             workspace=W256.ws), reps, flush)
+        gsp = graph_of(lambda: slc.sparse_decode(W256.q, W256.cache, W256.bt, W256.sl, y.prefix,
+                                                 y.window, y.budget, out=W256.out,
+                                                 workspace=W256.ws))
+        sp_graph = timed(gsp.replay, reps, flush)
+        dn = timed(lambda: slc.dense_decode(W256.q, W256.cache, W256.bt, W256.sl, out=W256.out,
+                                            workspace=W256.ws), max(5, reps // 4), flush)
+        sel256 = W256.sel[:, :, :y.budget]
+        k_score = timed(lambda: slc.score_pages(W256.q, W256.cache, W256.bt, W256.sl, y.prefix,
+                                                y.window, scores=W256.scores), reps, flush)
+        k_select = timed(lambda: slc.select_pages(W256.scores, W256.sl, y.prefix, y.window,
+                                                  y.budget, selected=sel256), reps, flush)
+        k_attend = timed(lambda: slc.sparse_attend(W256.q, W256.cache, W256.bt, W256.sl,
+                                                   y.prefix, y.window, sel256, out=W256.out,
+                                                   workspace=W256.ws), reps, flush)
+        db256, _, _ = algorithmic_bytes(y.seq_lens.tolist(), y.wl.hq, y.wl.hkv, y.wl.head_dim,
+                                        0, 0, 0, True)
+        sb = b256[1] + y.wl.batch * y.wl.hq * y.wl.head_dim * 2
+        ab = b256[2] + y.wl.batch * y.wl.hq * y.wl.head_dim * 6
+        best = min(sp, sp_graph)
+        also["decode256k"] = {
+            "workload": "B=4, ctx 262144, Hq 32 / Hkv 4, d 128, page 16, prefix 128, "
+                        "window 4096, budget 256 pages, 64 needles/seq",
+            "sparse_us": round(best * 1e3, 2), "sparse_us_eager": round(sp * 1e3, 2),
+            "sparse_us_graph": round(sp_graph * 1e3, 2), "dense_us": round(dn * 1e3, 2),
+            "speedup_vs_dense": round(dn / best, 2),
+            "algorithmic_bytes": b256[0],
+            "hbm_gbs": round(b256[0] / (best * 1e-3) / 1e9, 1),
+            "step_roofline_frac": round(b256[0] / (best * 1e-3) / 1e9 / peak, 4),
+            "dense_gbs": round(db256 / (dn * 1e-3) / 1e9, 1),
+            "kernels": {
+                "score_pages": {"us": round(k_score * 1e3, 2), "bytes": sb,
+                                "gbs": round(sb / (k_score * 1e-3) / 1e9, 1),
+                                "frac": round(sb / (k_score * 1e-3) / 1e9 / peak, 4),
+                                "traffic": traffic.get(("score_pages", "decode256k"))},
+                "select_pages": {"us": round(k_select * 1e3, 2)},
+                "sparse_attend": {"us": round(k_attend * 1e3, 2), "bytes": ab,
+                                  "gbs": round(ab / (k_attend * 1e-3) / 1e9, 1),
+                                  "frac": round(ab / (k_attend * 1e-3) / 1e9 / peak, 4),
+                                  "traffic": traffic.get(("sparse_attend", "decode256k"))}}}
+        assert slc.device_status() == 0
+
+    result = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": Wm, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": "decode64k: B=4, ctx 65536 (+1 token per step), Hq 32 / Hkv 4, d 128, "
+                        "page 16, prefix 128, window 1024, budget 128 pages, 64 needles/seq; "
+                        "step = kv_append + sparse_decode (score, select, attend, merge), "
+                        "CUDA graph",
+            "global_batch": B * world, "seq_len": int(L0[0]), "parallelism": "replicas",
+            "l2": "flushed (256 MiB write) before every timed step, outside its events"},
+        "hbm_gbs": round(step_bytes / (ms_per_step * 1e-3) / 1e9, 1),
+        "step_roofline": {"bound": "hbm", "achieved": round(step_bytes / (ms_per_step * 1e-3) / 1e9, 1),
+                          "peak": peak, "unit": "GB/s",
+                          "frac": round(step_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 4),
+                          "algorithmic_bytes": step_bytes},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": K * (1 + slc.KERNELS_PER_CALL["sparse_decode"]),
+        "clocks": clocks.summary(),
+        "timed_wall_s": round(t_wall, 4),
+        "also": also,
+    }
+    return result
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(seconds):
+    """The oracle, as it stands, on whole 64k decode steps (step 0 inputs),
+    repeated for about `seconds` of CPU time (at least once)."""
+    import oracle
+    import synth
+    wl = synth.WORKLOADS["decode64k"]
+    x = synth.make_inputs(wl, headroom_tokens=0)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.sparse_decode(x.q, x.k_cache, x.v_cache, x.block_table, x.seq_lens, x.prefix,
+                             x.window, x.budget)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or n >= 1000:
+            break
+    return {"value": round(el / n * 1e6, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "%d whole decode64k steps (B=4, 16 units; bounds rebuilt each step), "
+                      "single-threaded C fp64" % n}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: K timed steps, each one whole 64k
+    decode step on the host cores."""
+    import oracle
+    import synth
+    if rank != 0:
+        return None
+    wl = synth.WORKLOADS["decode64k"]
+    x = synth.make_inputs(wl, headroom_tokens=0)
+
+    def one():
+        oracle.sparse_decode(x.q, x.k_cache, x.v_cache, x.block_table, x.seq_lens, x.prefix,
+                             x.window, x.budget)
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    el = time.perf_counter() - t0
+    us = el / args.steps * 1e6
+    return {"metric": METRIC, "value": round(us, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1e3, 3),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": "decode64k: B=4, ctx 65536, Hq 32 / Hkv 4, d 128, page 16, "
+                                   "prefix 128, window 1024, budget 128 pages, 64 needles/seq",
+                       "global_batch": wl.batch, "seq_len": wl.context,
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(us, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": "%d whole decode64k steps" % args.steps},
+            "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    rank, world, local = rank_info()
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    res = run_ours(args, rank, world, local)
+    if rank == 0:
+        res["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

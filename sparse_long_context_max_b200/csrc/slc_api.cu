@@ -1,0 +1,318 @@
+// C ABI of libslc (declared in include/slc.h): argument validation,
+// workspace carving and kernel launches.  Validation happens before any
+// CUDA call, so argument errors launch nothing and need no GPU.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "slc_internal.h"
+
+// The device status word (SLC_STATUS_* bits), one per GPU that loads the
+// library; kernels receive its address.
+__device__ unsigned slc_status_word;
+
+namespace slc {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready;
+    int num_sms;
+    unsigned* status;
+};
+
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_mutex;
+thread_local char g_cuda_error[256];
+
+int note_cuda(cudaError_t e) {
+    snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),
+             cudaGetErrorString(e));
+    return SLC_ERR_CUDA;
+}
+
+// Per-device facts, looked up on the first call made with that device
+// current.
+int device_info(DeviceInfo** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return note_cuda(e);
+    if (dev < 0 || dev >= kMaxDevices) return SLC_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo& d = g_devices[dev];
+    if (!d.ready) {
+        e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return note_cuda(e);
+        e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), slc_status_word);
+        if (e != cudaSuccess) return note_cuda(e);
+        d.ready = true;
+    }
+    *out = &d;
+    return SLC_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int check_cache(const slc_cache_t* c) {
+    if (!c) return SLC_ERR_INVALID_ARG;
+    if (c->page_size != kPage) return SLC_ERR_UNSUPPORTED;
+    if (c->head_dim != 128 && c->head_dim != 256) return SLC_ERR_UNSUPPORTED;
+    if (c->num_kv_heads <= 0 || c->num_pages <= 0) return SLC_ERR_INVALID_ARG;
+    if (!c->k_cache || !c->v_cache || !c->meta) return SLC_ERR_INVALID_ARG;
+    if (!aligned16(c->k_cache) || !aligned16(c->v_cache) || !aligned16(c->meta))
+        return SLC_ERR_INVALID_ARG;
+    return SLC_OK;
+}
+
+int check_heads(const slc_cache_t* c, int hq) {
+    if (hq <= 0 || hq % c->num_kv_heads != 0) return SLC_ERR_INVALID_ARG;
+    const int g = hq / c->num_kv_heads;
+    if (g > kMaxGroup) return SLC_ERR_UNSUPPORTED;
+    return SLC_OK;
+}
+
+}  // namespace
+
+WorkspaceLayout workspace_layout(int batch, int hq, int hkv, int head_dim, int max_pages,
+                                 int budget) {
+    WorkspaceLayout w{};
+    const size_t units = (size_t)batch * hkv;
+    const size_t group = (size_t)(hq / hkv);
+    const size_t slots = units + kMaxAttendWarps;
+    size_t off = 0;
+    w.scores = off;
+    off = round_up(off + units * max_pages * sizeof(float), 256);
+    w.selected = off;
+    off = round_up(off + units * (size_t)(budget > 0 ? budget : 1) * sizeof(int32_t), 256);
+    w.part_acc = off;
+    off = round_up(off + slots * group * head_dim * sizeof(float), 256);
+    w.part_ml = off;
+    off = round_up(off + slots * group * sizeof(float2), 256);
+    w.total = off;
+    return w;
+}
+
+}  // namespace slc
+
+using namespace slc;
+
+extern "C" {
+
+const char* slc_error_string(int code) {
+    switch (code) {
+        case SLC_OK: return "ok";
+        case SLC_ERR_INVALID_ARG: return "invalid argument";
+        case SLC_ERR_UNSUPPORTED: return "unsupported shape";
+        case SLC_ERR_WORKSPACE: return "workspace too small";
+        case SLC_ERR_CUDA: return "CUDA error";
+        case SLC_ERR_DEVICE: return "device status fault";
+        default: return "unknown error";
+    }
+}
+
+const char* slc_last_cuda_error(void) { return g_cuda_error; }
+
+size_t slc_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                          int32_t head_dim, int32_t max_pages_per_seq, int32_t budget) {
+    if (batch < 0 || num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % num_kv_heads ||
+        num_q_heads / num_kv_heads > kMaxGroup || (head_dim != 128 && head_dim != 256) ||
+        max_pages_per_seq <= 0 || budget < 0)
+        return 0;
+    return workspace_layout(batch, num_q_heads, num_kv_heads, head_dim, max_pages_per_seq,
+                            budget)
+        .total;
+}
+
+int slc_kv_append(const slc_cache_t* cache, const void* k_new, const void* v_new,
+                  const int32_t* block_table, int32_t max_pages_per_seq,
+                  const int32_t* positions, int32_t batch, slc_stream_t stream) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if (batch < 0 || max_pages_per_seq <= 0) return SLC_ERR_INVALID_ARG;
+    if (batch == 0) return SLC_OK;
+    if (!k_new || !v_new || !block_table || !positions) return SLC_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new)) return SLC_ERR_INVALID_ARG;
+    DeviceInfo* dev;
+    if ((rc = device_info(&dev))) return rc;
+    KvAppendParams p{k_new,     v_new,     cache->k_cache,          cache->v_cache,
+                     cache->meta, block_table, positions,            dev->status,
+                     batch,     cache->num_kv_heads, max_pages_per_seq, cache->num_pages};
+    cudaError_t e = launch_kv_append(p, cache->head_dim, stream);
+    return e == cudaSuccess ? SLC_OK : note_cuda(e);
+}
+
+int slc_build_page_meta(const slc_cache_t* cache, const int32_t* block_table,
+                        int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                        slc_stream_t stream) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if (batch < 0 || max_pages_per_seq <= 0) return SLC_ERR_INVALID_ARG;
+    if (batch == 0) return SLC_OK;
+    if (!block_table || !seq_lens) return SLC_ERR_INVALID_ARG;
+    DeviceInfo* dev;
+    if ((rc = device_info(&dev))) return rc;
+    BuildMetaParams p{cache->k_cache, cache->meta, block_table, seq_lens, dev->status, batch,
+                      cache->num_kv_heads, max_pages_per_seq, cache->num_pages};
+    cudaError_t e = launch_build_meta(p, cache->head_dim, dev->num_sms, stream);
+    return e == cudaSuccess ? SLC_OK : note_cuda(e);
+}
+
+int slc_score_pages(const void* q, const slc_cache_t* cache, const int32_t* block_table,
+                    int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                    int32_t num_q_heads, int32_t prefix, int32_t window, float* scores,
+                    slc_stream_t stream) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if ((rc = check_heads(cache, num_q_heads))) return rc;
+    if (batch < 0 || max_pages_per_seq <= 0 || prefix < 0 || window < 0)
+        return SLC_ERR_INVALID_ARG;
+    if (batch == 0) return SLC_OK;
+    if (!q || !block_table || !seq_lens || !scores || !aligned16(q)) return SLC_ERR_INVALID_ARG;
+    DeviceInfo* dev;
+    if ((rc = device_info(&dev))) return rc;
+    ScoreParams p{q,     cache->meta, block_table, seq_lens, scores, dev->status, batch,
+                  num_q_heads, cache->num_kv_heads, num_q_heads / cache->num_kv_heads,
+                  max_pages_per_seq, cache->num_pages, prefix, window};
+    cudaError_t e = launch_score(p, cache->head_dim, dev->num_sms, stream);
+    return e == cudaSuccess ? SLC_OK : note_cuda(e);
+}
+
+int slc_select_pages(const float* scores, int32_t num_kv_heads, int32_t max_pages_per_seq,
+                     const int32_t* seq_lens, int32_t batch, int32_t prefix, int32_t window,
+                     int32_t budget, int32_t* selected, slc_stream_t stream) {
+    if (batch < 0 || num_kv_heads <= 0 || max_pages_per_seq <= 0 || prefix < 0 ||
+        window < 0 || budget < 0)
+        return SLC_ERR_INVALID_ARG;
+    if (max_pages_per_seq > kMaxCandidates) return SLC_ERR_UNSUPPORTED;
+    if (batch == 0 || budget == 0) return SLC_OK;
+    if (!scores || !seq_lens || !selected) return SLC_ERR_INVALID_ARG;
+    DeviceInfo* dev;
+    int rc;
+    if ((rc = device_info(&dev))) return rc;
+    SelectParams p{scores, seq_lens, selected, dev->status, batch, num_kv_heads,
+                   max_pages_per_seq, prefix, window, budget};
+    cudaError_t e = launch_select(p, stream);
+    return e == cudaSuccess ? SLC_OK : note_cuda(e);
+}
+
+// mode: 0 dense, 1 sparse (score + select + attend), 2 sparse attend over
+// the caller's selection in `selected_out`.
+static int decode(int mode, const void* q, const slc_cache_t* cache,
+                  const int32_t* block_table, int32_t max_pages_per_seq,
+                  const int32_t* seq_lens, int32_t batch, int32_t num_q_heads, int32_t prefix,
+                  int32_t window, int32_t budget, float scale, float* out,
+                  int32_t* selected_out, void* workspace, size_t workspace_bytes,
+                  cudaStream_t stream) {
+    const bool sparse = mode != 0;
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if ((rc = check_heads(cache, num_q_heads))) return rc;
+    if (batch < 0 || max_pages_per_seq <= 0 || prefix < 0 || window < 0 || budget < 0)
+        return SLC_ERR_INVALID_ARG;
+    if (sparse && max_pages_per_seq > kMaxCandidates) return SLC_ERR_UNSUPPORTED;
+    if (!(scale == scale) || isinf(scale)) return SLC_ERR_INVALID_ARG;
+    if (batch == 0) return SLC_OK;
+    if (!q || !block_table || !seq_lens || !out || !workspace) return SLC_ERR_INVALID_ARG;
+    if (mode == 2 && budget > 0 && !selected_out) return SLC_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return SLC_ERR_INVALID_ARG;
+    const int hkv = cache->num_kv_heads, D = cache->head_dim;
+    const WorkspaceLayout w =
+        workspace_layout(batch, num_q_heads, hkv, D, max_pages_per_seq, sparse ? budget : 0);
+    if (workspace_bytes < w.total) return SLC_ERR_WORKSPACE;
+    DeviceInfo* dev;
+    if ((rc = device_info(&dev))) return rc;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (scale <= 0.f) scale = 1.f / sqrtf((float)D);
+    int32_t* sel = selected_out ? selected_out : reinterpret_cast<int32_t*>(ws + w.selected);
+    cudaError_t e = cudaSuccess;
+    if (mode == 1 && budget > 0) {
+        float* scores = reinterpret_cast<float*>(ws + w.scores);
+        ScoreParams sp{q,           cache->meta, block_table, seq_lens,
+                       scores,      dev->status, batch,       num_q_heads,
+                       hkv,         num_q_heads / hkv,        max_pages_per_seq,
+                       cache->num_pages, prefix,  window};
+        e = launch_score(sp, D, dev->num_sms, stream);
+        if (e != cudaSuccess) return note_cuda(e);
+        SelectParams lp{scores, seq_lens, sel, dev->status, batch, hkv, max_pages_per_seq,
+                        prefix, window, budget};
+        e = launch_select(lp, stream);
+        if (e != cudaSuccess) return note_cuda(e);
+    }
+    AttendParams ap{};
+    ap.q = q;
+    ap.k_cache = cache->k_cache;
+    ap.v_cache = cache->v_cache;
+    ap.block_table = block_table;
+    ap.seq_lens = seq_lens;
+    ap.selected = sel;
+    ap.part_acc = reinterpret_cast<float*>(ws + w.part_acc);
+    ap.part_ml = reinterpret_cast<float2*>(ws + w.part_ml);
+    ap.out = out;
+    ap.status = dev->status;
+    ap.batch = batch;
+    ap.hq = num_q_heads;
+    ap.hkv = hkv;
+    ap.group = num_q_heads / hkv;
+    ap.max_pages = max_pages_per_seq;
+    ap.num_pages = cache->num_pages;
+    ap.sparse = sparse ? 1 : 0;
+    ap.prefix = prefix;
+    ap.window = window;
+    ap.budget = sparse ? budget : 0;
+    ap.scale_log2 = scale * 1.4426950408889634f;
+    e = launch_attend(ap, D, dev->num_sms, stream, nullptr);
+    return e == cudaSuccess ? SLC_OK : note_cuda(e);
+}
+
+int slc_sparse_decode(const void* q, const slc_cache_t* cache, const int32_t* block_table,
+                      int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                      int32_t num_q_heads, int32_t prefix, int32_t window, int32_t budget,
+                      float scale, float* out, int32_t* selected_out, void* workspace,
+                      size_t workspace_bytes, slc_stream_t stream) {
+    return decode(1, q, cache, block_table, max_pages_per_seq, seq_lens, batch, num_q_heads,
+                  prefix, window, budget, scale, out, selected_out, workspace, workspace_bytes,
+                  stream);
+}
+
+int slc_sparse_attend(const void* q, const slc_cache_t* cache, const int32_t* block_table,
+                      int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                      int32_t num_q_heads, int32_t prefix, int32_t window, int32_t budget,
+                      const int32_t* selected, float scale, float* out, void* workspace,
+                      size_t workspace_bytes, slc_stream_t stream) {
+    return decode(2, q, cache, block_table, max_pages_per_seq, seq_lens, batch, num_q_heads,
+                  prefix, window, budget, scale, out, const_cast<int32_t*>(selected), workspace,
+                  workspace_bytes, stream);
+}
+
+int slc_dense_decode(const void* q, const slc_cache_t* cache, const int32_t* block_table,
+                     int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                     int32_t num_q_heads, float scale, float* out, void* workspace,
+                     size_t workspace_bytes, slc_stream_t stream) {
+    return decode(0, q, cache, block_table, max_pages_per_seq, seq_lens, batch,
+                  num_q_heads, 0, 0, 0, scale, out, nullptr, workspace, workspace_bytes,
+                  stream);
+}
+
+int slc_device_status(int32_t* status, slc_stream_t stream) {
+    if (!status) return SLC_ERR_INVALID_ARG;
+    DeviceInfo* dev;
+    int rc;
+    if ((rc = device_info(&dev))) return rc;
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return note_cuda(e);
+    unsigned v = 0;
+    e = cudaMemcpy(&v, dev->status, sizeof v, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return note_cuda(e);
+    e = cudaMemset(dev->status, 0, sizeof v);
+    if (e != cudaSuccess) return note_cuda(e);
+    *status = (int32_t)v;
+    return SLC_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,400 @@
+// Split-KV flash-decode over a paged bf16 KV cache, and the log-sum-exp
+// merge of the split partials.
+//
+// Each (sequence, kv head) unit attends a list of logical pages:
+//   dense   all pages [0, n)                       (every key, each step:
+//           "Hybrid LLM Decoding 2.2x Faster at 256k, No Retraining",
+//           section "The remaining full-attention layers are the
+//           long-context bill")
+//   sparse  prefix pages, then the selected pages, then window pages
+//           (same article, section "The method: sliding window + prefix +
+//           query-aware pages, searched per layer")
+// The lists of all units are concatenated and cut into equal chunks, one per
+// warp of a persistent grid, so work is balanced by pages whatever the
+// sequence lengths.  A chunk that spans unit boundaries yields one partial
+// (running max m, sum l, unnormalised accumulator) per unit piece, stored in
+// slot (unit + chunk), which is unique.  The merge kernel combines a unit's
+// partials: out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k.
+//
+// Per warp, pages stream through a private ring of shared-memory stages,
+// each filled by two 1-D bulk copies (TMA engine: the K and V tiles of one
+// (page, kv head) are contiguous, 32*D bytes each) completing on an
+// mbarrier.  The group's query heads (G <= 8) and the 16 tokens of a page
+// are contracted on tensor cores with mma.sync m16n8k16 (bf16 in, fp32
+// accumulate):
+//   S   = Q K^T : A = Q (heads padded to 16 rows), B = K^T, 16 mma per page
+//   O^T += V^T P^T : A = V^T (16 dims per m-block), B = P^T (8 heads)
+// P is split into bf16 hi + lo parts (two mma per m-block) so the weights
+// carry ~16 mantissa bits.  The head_dim contraction index is permuted so
+// that each thread reads 16-byte vectors: logical k-step 2m / 2m+1 of thread
+// (r, c) covers physical dims 8*(c+4m)..8*(c+4m)+7, identically for Q and K.
+// For P V, thread (r, c) owns dims (D/8)*r .. (D/8)*r + D/8 - 1, read as
+// 16-byte vectors and paired across tokens with byte permutes.
+#include "slc_internal.h"
+
+namespace slc {
+
+namespace {
+
+constexpr uint32_t kWaitLimit = 1u << 22;  // bounded mbarrier polls
+
+struct Ring {
+    uint8_t* tiles;  // STAGES x (K tile, V tile)
+    uint64_t* bars;  // STAGES
+    int* nvalid;     // STAGES
+};
+
+// Logical page of list position i of a unit (and whether it is sane).
+__device__ __forceinline__ int list_page(const AttendParams& p, int u, const PageRanges& r,
+                                         int nsel, int i, bool* ok) {
+    *ok = true;
+    if (!p.sparse || i < r.np) return i;
+    if (i < r.np + nsel) {
+        const int j = p.selected[(long long)u * p.budget + (i - r.np)];
+        if (j < r.np || j >= r.ws) {
+            *ok = false;
+            return 0;
+        }
+        return j;
+    }
+    return r.ws + (i - r.np - nsel);
+}
+
+template <int D>
+__device__ __forceinline__ void issue_page(const AttendParams& p, const Ring& ring, int stage,
+                                           int u, int b, int h, const PageRanges& r, int nsel,
+                                           int L, int i) {
+    constexpr uint32_t TILE = kPage * D * 2;
+    bool ok;
+    const int j = list_page(p, u, r, nsel, i, &ok);
+    int phys = 0, nv = 0;
+    if (!ok) {
+        atomicOr(p.status, SLC_STATUS_BAD_SELECTION);
+    } else {
+        phys = p.block_table[(long long)b * p.max_pages + j];
+        if (phys < 0 || phys >= p.num_pages) {
+            atomicOr(p.status, SLC_STATUS_BAD_PAGE);
+            phys = 0;
+        } else {
+            nv = min(kPage, L - j * kPage);
+        }
+    }
+    ring.nvalid[stage] = nv;
+    uint64_t* bar = ring.bars + stage;
+    mbar_arrive_expect_tx(bar, 2 * TILE);
+    const long long off = ((long long)phys * p.hkv + h) * (kPage * D);
+    uint8_t* dst = ring.tiles + stage * 2 * TILE;
+    bulk_g2s(dst, static_cast<const __nv_bfloat16*>(p.k_cache) + off, TILE, bar);
+    bulk_g2s(dst + TILE, static_cast<const __nv_bfloat16*>(p.v_cache) + off, TILE, bar);
+}
+
+// Process list positions [i0, i1) of unit u; write the partial to `slot`.
+// `it` counts ring uses of this warp (stage = it % STAGES).  Returns false
+// if a bounded wait gave up (the warp then stops).
+template <int D, int STAGES>
+__device__ bool attend_piece(const AttendParams& p, const Ring& ring, uint32_t& it, int u,
+                             int i0, int i1, long long slot) {
+    constexpr int TILE_W = kPage * D / 2;  // 32-bit words per tile
+    constexpr int ROW_W = D / 2;           // words per token row
+    constexpr int KS = D / 16;             // k-steps of Q K^T, m-blocks of V^T P^T
+    const int lane = threadIdx.x & 31;
+    const int r_ = lane >> 2, c_ = lane & 3;
+    const int b = u / p.hkv, h = u % p.hkv;
+    const int G = p.group;
+    const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
+    const PageRanges r = page_ranges(L, p.prefix, p.window);
+    const int nsel = p.sparse ? min(p.budget, r.ws - r.np) : 0;
+    const int npg = i1 - i0;
+
+    // query fragments (rows >= G and rows 8..15 are zero)
+    uint32_t qa[KS][2];
+    if (r_ < G) {
+        const uint4* qrow = reinterpret_cast<const uint4*>(
+            static_cast<const __nv_bfloat16*>(p.q) + ((long long)b * p.hq + h * G + r_) * D);
+#pragma unroll
+        for (int m = 0; m < D / 32; ++m) {
+            const uint4 v = qrow[c_ + 4 * m];
+            qa[2 * m][0] = v.x;
+            qa[2 * m][1] = v.y;
+            qa[2 * m + 1][0] = v.z;
+            qa[2 * m + 1][1] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < KS; ++k) qa[k][0] = qa[k][1] = 0u;
+    }
+
+    __syncwarp();  // the previous piece's reads of the ring are done
+    if (lane == 0) {
+        fence_proxy_async_smem();
+        for (int k = 0; k < STAGES && k < npg; ++k)
+            issue_page<D>(p, ring, (it + k) % STAGES, u, b, h, r, nsel, L, i0 + k);
+    }
+    __syncwarp();
+
+    float m_run = -INFINITY, l_run = 0.f;
+    float acc[KS][4];
+#pragma unroll
+    for (int i = 0; i < KS; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+
+    for (int k = 0; k < npg; ++k) {
+        const uint32_t use = it + k;
+        const int stage = use % STAGES;
+        if (!mbar_wait_bounded(ring.bars + stage, (use / STAGES) & 1u, kWaitLimit)) {
+            // give up: record it, drain this warp's copies in flight, stop
+            if (lane == 0) {
+                atomicOr(p.status, SLC_STATUS_WAIT_TIMEOUT);
+                for (int kk = k; kk < npg && kk < k + STAGES; ++kk) {
+                    const uint32_t u2 = it + kk;
+                    mbar_wait_bounded(ring.bars + u2 % STAGES, (u2 / STAGES) & 1u, kWaitLimit);
+                }
+            }
+            __syncwarp();
+            return false;
+        }
+        const uint32_t* Kw = reinterpret_cast<const uint32_t*>(ring.tiles) + stage * 2 * TILE_W;
+        const uint32_t* Vw = Kw + TILE_W;
+        const int nv = ring.nvalid[stage];
+
+        // S = Q K^T for tokens nb*8 + (0..7)
+        float s[2][4];
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) {
+            s[nb][0] = s[nb][1] = s[nb][2] = s[nb][3] = 0.f;
+            const uint32_t* krow = Kw + (nb * 8 + r_) * ROW_W;
+#pragma unroll
+            for (int m = 0; m < D / 32; ++m) {
+                const uint4 kv = lds128(krow + (c_ + 4 * m) * 4);
+                mma_bf16(s[nb], qa[2 * m][0], 0u, qa[2 * m][1], 0u, kv.x, kv.y);
+                mma_bf16(s[nb], qa[2 * m + 1][0], 0u, qa[2 * m + 1][1], 0u, kv.z, kv.w);
+            }
+        }
+        // this thread: head r_, tokens 2c, 2c+1, 8+2c, 9+2c
+        const int t0 = 2 * c_;
+        float x[4];
+        x[0] = t0 < nv ? s[0][0] * p.scale_log2 : -INFINITY;
+        x[1] = t0 + 1 < nv ? s[0][1] * p.scale_log2 : -INFINITY;
+        x[2] = t0 + 8 < nv ? s[1][0] * p.scale_log2 : -INFINITY;
+        x[3] = t0 + 9 < nv ? s[1][1] * p.scale_log2 : -INFINITY;
+        float pmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+        pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 1));
+        pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 2));
+        const float m_new = fmaxf(m_run, pmax);
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+        const float alpha = ex2(m_run - m_use);
+        float pr[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pr[e] = ex2(x[e] - m_use);
+        l_run = l_run * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
+        m_run = m_new;
+        const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * c_);
+        const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * c_ + 4);
+#pragma unroll
+        for (int i = 0; i < KS; ++i) {
+            acc[i][0] *= a0;
+            acc[i][1] *= a1;
+            acc[i][2] *= a0;
+            acc[i][3] *= a1;
+        }
+        // P^T fragments (tokens 2c,2c+1 / 2c+8,2c+9 of head r_), hi + lo
+        const uint32_t bh0 = pack_bf16x2(pr[0], pr[1]);
+        const uint32_t bh1 = pack_bf16x2(pr[2], pr[3]);
+        const uint32_t bl0 = pack_bf16x2(pr[0] - bf16_lo(bh0), pr[1] - bf16_hi(bh0));
+        const uint32_t bl1 = pack_bf16x2(pr[2] - bf16_lo(bh1), pr[3] - bf16_hi(bh1));
+
+        // V rows of tokens 2c, 2c+1, 2c+8, 2c+9, dims (D/8)*r_ .. +D/8
+        constexpr int WPT = D / 16;  // words per token per thread
+        uint32_t vw[4][WPT];
+#pragma unroll
+        for (int tt = 0; tt < 4; ++tt) {
+            const int tok = t0 + (tt & 1) + (tt >> 1) * 8;
+            const uint32_t* vrow = Vw + tok * ROW_W + WPT * r_;
+#pragma unroll
+            for (int q4 = 0; q4 < WPT / 4; ++q4) {
+                const uint4 v = lds128(vrow + 4 * q4);
+                const bool live = tok < nv;  // zero slots past the length (may hold NaN)
+                vw[tt][4 * q4 + 0] = live ? v.x : 0u;
+                vw[tt][4 * q4 + 1] = live ? v.y : 0u;
+                vw[tt][4 * q4 + 2] = live ? v.z : 0u;
+                vw[tt][4 * q4 + 3] = live ? v.w : 0u;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < KS; ++i) {
+            const uint32_t a0r = __byte_perm(vw[0][i], vw[1][i], 0x5410);
+            const uint32_t a1r = __byte_perm(vw[0][i], vw[1][i], 0x7632);
+            const uint32_t a2r = __byte_perm(vw[2][i], vw[3][i], 0x5410);
+            const uint32_t a3r = __byte_perm(vw[2][i], vw[3][i], 0x7632);
+            mma_bf16(acc[i], a0r, a1r, a2r, a3r, bh0, bh1);
+            mma_bf16(acc[i], a0r, a1r, a2r, a3r, bl0, bl1);
+        }
+        __syncwarp();
+        if (lane == 0 && k + STAGES < npg) {
+            fence_proxy_async_smem();
+            issue_page<D>(p, ring, stage, u, b, h, r, nsel, L, i0 + k + STAGES);
+        }
+    }
+    it += npg;
+
+    // partial: (m, l) of head r_, accumulators of heads 2c, 2c+1
+    float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
+    if (c_ == 0 && r_ < G) p.part_ml[slot * G + r_] = make_float2(m_run, l_tot);
+    constexpr int DPT = D / 8;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const int head = 2 * c_ + hh;
+        if (head < G) {
+            float4* dst =
+                reinterpret_cast<float4*>(p.part_acc + (slot * G + head) * D + DPT * r_);
+#pragma unroll
+            for (int i2 = 0; i2 < KS / 2; ++i2)
+                dst[i2] = make_float4(acc[2 * i2][hh], acc[2 * i2][2 + hh], acc[2 * i2 + 1][hh],
+                                      acc[2 * i2 + 1][2 + hh]);
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ int list_len(const AttendParams& p, int b) {
+    const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
+    const PageRanges r = page_ranges(L, p.prefix, p.window);
+    if (!p.sparse) return r.n;
+    return r.np + min(p.budget, r.ws - r.np) + (r.n - r.ws);
+}
+
+template <int D, int NW, int STAGES>
+__global__ void __launch_bounds__(NW * 32) attend_kernel(AttendParams p) {
+    constexpr int TILE = kPage * D * 2;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    Ring ring;
+    ring.tiles = smem + warp * STAGES * 2 * TILE;
+    ring.bars = reinterpret_cast<uint64_t*>(smem + NW * STAGES * 2 * TILE) + warp * STAGES;
+    ring.nvalid = reinterpret_cast<int*>(smem + NW * STAGES * 2 * TILE + NW * STAGES * 8) +
+                  warp * STAGES;
+    if (lane == 0) {
+        for (int s = 0; s < STAGES; ++s) mbar_init(ring.bars + s, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    const int gw = blockIdx.x * NW + warp;
+    auto len_of = [&](int b) { return list_len(p, b); };
+    const long long total = total_units(p.batch, p.hkv, len_of);
+    const long long cpp = (total + p.total_warps - 1) / p.total_warps;
+    long long s = (long long)gw * cpp;
+    const long long e = min(total, s + cpp);
+    if (s >= e) return;
+    int u;
+    long long ustart;
+    locate_unit(s, p.batch, p.hkv, len_of, &u, &ustart);
+    uint32_t it = 0;
+    while (s < e) {
+        const int len = list_len(p, u / p.hkv);
+        if (len == 0) {
+            ++u;
+            continue;
+        }
+        const int i0 = (int)(s - ustart);
+        const int i1 = (int)(min(e, ustart + len) - ustart);
+        if (!attend_piece<D, STAGES>(p, ring, it, u, i0, i1, (long long)u + gw)) return;
+        s = ustart + len;
+        ustart = s;
+        ++u;
+    }
+}
+
+// One CTA per unit: combine the unit's partials (slots unit + chunk).
+template <int D>
+__global__ void __launch_bounds__(256) merge_kernel(AttendParams p) {
+    const int u = blockIdx.x;
+    const int b = u / p.hkv, h = u % p.hkv;
+    const int G = p.group;
+    __shared__ long long sh_off;
+    __shared__ long long sh_total;
+    if (threadIdx.x < 32) {
+        // offset of unit u in the concatenated lists, and the total
+        auto len_of = [&](int bb) { return list_len(p, bb); };
+        const long long total = total_units(p.batch, p.hkv, len_of);
+        long long base = 0;
+        for (int b0 = 0; b0 < b; b0 += 32) {
+            const int bb = b0 + threadIdx.x;
+            long long c = bb < b ? (long long)list_len(p, bb) * p.hkv : 0;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+            base += c;
+        }
+        if (threadIdx.x == 0) {
+            sh_off = base + (long long)h * list_len(p, b);
+            sh_total = total;
+        }
+    }
+    __syncthreads();
+    const int len = list_len(p, b);
+    const long long cpp = (sh_total + p.total_warps - 1) / p.total_warps;
+    const long long k0 = len > 0 ? sh_off / cpp : 0;
+    const long long k1 = len > 0 ? (sh_off + len - 1) / cpp : -1;
+    constexpr int V4 = D / 4;
+    for (int item = threadIdx.x; item < G * V4; item += blockDim.x) {
+        const int g = item / V4, d4 = item % V4;
+        float M = -INFINITY;
+        for (long long k = k0; k <= k1; ++k) M = fmaxf(M, p.part_ml[(u + k) * G + g].x);
+        const float Mu = M == -INFINITY ? 0.f : M;
+        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+        float den = 0.f;
+        for (long long k = k0; k <= k1; ++k) {
+            const float2 ml = p.part_ml[(u + k) * G + g];
+            const float w = ex2(ml.x - Mu);
+            const float4 a = reinterpret_cast<const float4*>(p.part_acc + ((u + k) * G + g) * D)[d4];
+            num.x = fmaf(w, a.x, num.x);
+            num.y = fmaf(w, a.y, num.y);
+            num.z = fmaf(w, a.z, num.z);
+            num.w = fmaf(w, a.w, num.w);
+            den = fmaf(w, ml.y, den);
+        }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        reinterpret_cast<float4*>(p.out + ((long long)b * p.hq + h * G + g) * D)[d4] =
+            make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+    }
+}
+
+template <int D, int NW, int STAGES>
+constexpr int attend_smem() {
+    return NW * STAGES * (2 * kPage * D * 2 + 8 + 4);
+}
+
+template <int D, int NW, int STAGES>
+cudaError_t run(AttendParams p, int num_sms, cudaStream_t stream, int* launched) {
+    constexpr int smem = attend_smem<D, NW, STAGES>();
+    static int occ = 0;
+    if (occ == 0) {
+        cudaError_t e = cudaFuncSetAttribute(attend_kernel<D, NW, STAGES>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, attend_kernel<D, NW, STAGES>,
+                                                          NW * 32, smem);
+        if (e != cudaSuccess) return e;
+        if (occ < 1) occ = 1;
+    }
+    int blocks = num_sms * occ;
+    if (blocks * NW > kMaxAttendWarps) blocks = kMaxAttendWarps / NW;
+    p.total_warps = blocks * NW;
+    attend_kernel<D, NW, STAGES><<<blocks, NW * 32, smem, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    merge_kernel<D><<<p.batch * p.hkv, 256, 0, stream>>>(p);
+    if (launched) *launched += 2;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attend(AttendParams p, int head_dim, int num_sms, cudaStream_t stream,
+                          int* launched) {
+    if (p.batch * p.hkv == 0) return cudaSuccess;
+    if (head_dim == 128) return run<128, 4, 3>(p, num_sms, stream, launched);
+    return run<256, 4, 3>(p, num_sms, stream, launched);
+}
+
+}  // namespace slc

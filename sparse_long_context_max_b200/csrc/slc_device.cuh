@@ -1,0 +1,194 @@
+// Device-side helpers shared by the sm_100a kernels of libslc.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/slc.h"
+
+namespace slc {
+
+constexpr int kPage = 16;        // tokens per page
+constexpr int kMaxGroup = 8;     // query heads per kv head handled per warp
+constexpr int kMaxCandidates = 32768;
+
+// ---------------------------------------------------------------- ranges
+// Page ranges of one sequence of L tokens (see include/slc.h):
+// n pages, prefix [0, np), candidates [np, ws), window [ws, n).
+struct PageRanges {
+    int n, np, ws;
+};
+
+__device__ __forceinline__ PageRanges page_ranges(int L, int prefix, int window) {
+    PageRanges r;
+    r.n = L > 0 ? (L + kPage - 1) / kPage : 0;
+    r.np = min((prefix + kPage - 1) / kPage, r.n);
+    int ws = r.n;
+    if (window > 0) ws = max(L - window, 0) / kPage;
+    r.ws = min(max(ws, r.np), r.n);
+    return r;
+}
+
+// Sequence length with the device-side range check applied.
+__device__ __forceinline__ int checked_len(const int32_t* seq_lens, int b, int max_pages,
+                                           unsigned* status) {
+    int L = seq_lens[b];
+    if (L < 0 || L > max_pages * kPage) {
+        atomicOr(status, SLC_STATUS_BAD_LENGTH);
+        L = L < 0 ? 0 : max_pages * kPage;
+    }
+    return L;
+}
+
+// ---------------------------------------------------------------- bf16
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ---------------------------------------------------------------- warp
+__device__ __forceinline__ int warp_incl_scan(int v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int t = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += t;
+    }
+    return v;
+}
+
+// Locate global index g among segments whose sizes are count(b) * hkv,
+// b = 0..batch-1 (each sequence contributes hkv equal units).  Returns the
+// unit u = b * hkv + h containing g and the unit's start offset.  Warp-wide:
+// every lane must call it with the same g; count(b) must be warp-uniform
+// per b.  If g is past the end, returns u = batch * hkv.
+template <class CountFn>
+__device__ __forceinline__ void locate_unit(long long g, int batch, int hkv, CountFn count,
+                                            int* unit_out, long long* start_out) {
+    const int lane = threadIdx.x & 31;
+    long long base = 0;
+    for (int b0 = 0; b0 < batch; b0 += 32) {
+        int b = b0 + lane;
+        int c = b < batch ? count(b) : 0;
+        long long seg = (long long)c * hkv;
+        // inclusive scan of seg (64-bit via two 32-bit halves is overkill:
+        // segment sizes stay below 2^31 per chunk of 32 sequences)
+        int s32 = warp_incl_scan((int)seg);
+        long long incl = base + s32;
+        unsigned hit = __ballot_sync(0xffffffffu, b < batch && incl > g);
+        if (hit) {
+            int l = __ffs(hit) - 1;
+            long long excl = __shfl_sync(0xffffffffu, incl - seg, l);
+            int cb = __shfl_sync(0xffffffffu, c, l);
+            int h = (int)((g - excl) / cb);
+            *unit_out = (b0 + l) * hkv + h;
+            *start_out = excl + (long long)h * cb;
+            return;
+        }
+        base += __shfl_sync(0xffffffffu, s32, 31);
+    }
+    *unit_out = batch * hkv;
+    *start_out = base;
+}
+
+// Total of count(b) * hkv over all sequences (warp-wide).
+template <class CountFn>
+__device__ __forceinline__ long long total_units(int batch, int hkv, CountFn count) {
+    const int lane = threadIdx.x & 31;
+    long long tot = 0;
+    for (int b0 = 0; b0 < batch; b0 += 32) {
+        int b = b0 + lane;
+        long long c = b < batch ? (long long)count(b) * hkv : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        tot += c;
+    }
+    return tot;
+}
+
+// ---------------------------------------------------------------- PTX
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: gives up after `limit` polls (each try_wait may suspend the
+// thread for a hardware-defined interval) and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  uint32_t limit) {
+    for (uint32_t i = 0; i < limit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+// 1-D bulk copy global -> shared (TMA engine), completion counted on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+        "[%3];" ::"r"(smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(const void* p) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(smem_addr(p)));
+    return v;
+}
+
+// D += A * B, m16n8k16, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 2^x on the SFU (PTX ex2.approx.ftz.f32); ex2(-inf) = +0.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+}  // namespace slc

@@ -1,0 +1,304 @@
+"""CUDA path against the fp64 oracle, element by element, on seeded inputs.
+
+Bars: page metadata bit-exact; page selection identical except pages whose
+oracle score is within 1e-4 (relative) of the k-th score; outputs within
+2e-3 max-abs of the oracle attending the GPU's own selection."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_util import (Dev, check_needles, check_output, check_selection, slice_batch)
+
+pytestmark = pytest.mark.gpu
+
+W = synth.WORKLOADS
+
+
+def small(B, hq, hkv, D, lens, prefix=0, window=0, budget=0, layout="shuffled", seed=3,
+          fill="zero", needles=0, headroom=0):
+    wl = synth.Workload(name="t", batch=B, hq=hq, hkv=hkv, head_dim=D, prefix=prefix,
+                        window=window, budget=budget, needles=needles, seed=seed,
+                        context=max(lens), layout=layout)
+    return synth.make_inputs(wl, lens_override=lens, fill=fill, headroom_tokens=headroom)
+
+
+def meta_matches_oracle(d):
+    x = d.x
+    kmin, kmax = oracle.page_bounds(x.k_cache, x.block_table, x.seq_lens)
+    meta = d.cache.meta.cpu().double().numpy()  # [pages][Hkv][2][D]
+    bt = x.block_table.numpy()
+    for b, L in enumerate(x.seq_lens.tolist()):
+        n = -(-L // 16)
+        phys = bt[b, :n]
+        got_min = meta[phys, :, 0, :].transpose(1, 0, 2)  # [Hkv][n][D]
+        got_max = meta[phys, :, 1, :].transpose(1, 0, 2)
+        np.testing.assert_array_equal(got_min, kmin[b, :, :n])
+        np.testing.assert_array_equal(got_max, kmax[b, :, :n])
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    return Dev(synth.make_inputs(W["tiny"]))
+
+
+# ------------------------------------------------------------------ metadata
+
+def test_build_page_meta_exact(tiny):
+    meta_matches_oracle(tiny)
+
+
+def test_build_page_meta_exact_ragged_lengths_nan_slots():
+    x = small(5, 8, 4, 256, [1, 16, 17, 250, 1000], fill="nan", seed=7)
+    meta_matches_oracle(Dev(x))
+
+
+def test_kv_append_matches_rebuild_and_oracle():
+    import sparse_long_context_max_b200 as slc
+    x = small(3, 8, 2, 128, [30, 47, 16], seed=9, headroom=40)
+    d = Dev(x)
+    lens = x.seq_lens.clone()
+    for step in range(40):
+        kn = torch.randn((3, 2, 128), generator=torch.Generator().manual_seed(step)).to(torch.bfloat16)
+        vn = torch.randn((3, 2, 128), generator=torch.Generator().manual_seed(99 + step)).to(torch.bfloat16)
+        slc.kv_append(d.cache, kn.cuda(), vn.cuda(), d.bt, lens.cuda())
+        for b in range(3):
+            L = int(lens[b])
+            phys = int(x.block_table[b, L // 16])
+            x.k_cache[phys, :, L % 16] = kn[b]
+            x.v_cache[phys, :, L % 16] = vn[b]
+        lens += 1
+    torch.cuda.synchronize()
+    assert slc.device_status() == 0
+    # the appended tokens landed where the host put them
+    assert torch.equal(d.k.cpu(), x.k_cache)
+    assert torch.equal(d.v.cpu(), x.v_cache)
+    x.seq_lens = lens
+    d.sl = lens.cuda()
+    incremental = d.cache.meta.clone()
+    meta_matches_oracle(d)
+    slc.build_page_meta(d.cache, d.bt, d.sl)
+    rebuilt = d.cache.meta
+    used = sorted(set(int(p) for b in range(3) for p in x.block_table[b, : -(-int(lens[b]) // 16)]))
+    assert torch.equal(incremental[used].float(), rebuilt[used].float())
+
+
+# ------------------------------------------------------------------ scoring
+
+def test_scores_match_oracle_and_bound(tiny):
+    import sparse_long_context_max_b200 as slc
+    x = tiny.x
+    s = slc.score_pages(tiny.q, tiny.cache, tiny.bt, tiny.sl, x.prefix, x.window).cpu().double().numpy()
+    kmin, kmax = oracle.page_bounds(x.k_cache, x.block_table, x.seq_lens)
+    so = oracle.page_scores(x.q, kmin, kmax, x.seq_lens, x.prefix, x.window)
+    cand = ~np.isnan(so)
+    assert cand.sum() == 2 * (240 - 4)
+    scale = np.abs(so[cand]).max()
+    assert np.abs(s[cand] - so[cand]).max() <= 2e-6 * scale
+    # the bound never drops below the best group logit of the page
+    G = 4
+    for h in range(2):
+        for j in range(4, 240):
+            phys = int(x.block_table[0, j])
+            k = x.k_cache[phys, h].double()
+            q = x.q[0, h * G:(h + 1) * G].double()
+            best = (q @ k.T).sum(0).max().item()
+            assert s[0, h, j] >= best - 1e-5 * abs(best) - 1e-4
+
+
+def test_select_exact_on_given_scores():
+    import sparse_long_context_max_b200 as slc
+    rng = np.random.default_rng(0)
+    for ncand, budget, ties in [(50, 7, True), (4000, 128, True), (16120, 256, False),
+                                (16120, 256, True), (30000, 512, True), (9, 3, True)]:
+        B, hkv = 2, 3
+        L = 16 * (ncand + 2)
+        P, Wn = 16, 16
+        scores = np.full((B, hkv, ncand + 2), np.nan, dtype=np.float32)
+        if ties:
+            vals = rng.integers(-20, 20, size=(B, hkv, ncand)).astype(np.float32)
+        else:
+            vals = rng.standard_normal((B, hkv, ncand)).astype(np.float32) * 100
+        scores[:, :, 1:ncand + 1] = vals
+        sl = torch.tensor([L, L], dtype=torch.int32)
+        sel = slc.select_pages(torch.from_numpy(scores).cuda(), sl.cuda(), P, Wn, budget)
+        want, _ = oracle.select_pages(scores.astype(np.float64), sl, P, Wn, budget)
+        np.testing.assert_array_equal(sel.cpu().numpy(), want)
+
+
+# ------------------------------------------------------------------ decode
+
+def test_tiny_sparse_parity(tiny):
+    x = tiny.x
+    out, sel = tiny.sparse()
+    check_selection(x, sel, x.prefix, x.window, x.budget)
+    check_needles(x, sel)
+    check_output(x, out, x.prefix, x.window, sel)
+
+
+def test_tiny_dense_parity(tiny):
+    check_output(tiny.x, tiny.dense(), 0, 0, None, dense=True)
+
+
+def test_coverage_equals_dense(tiny):
+    x = tiny.x
+    dense = tiny.dense()
+    out, sel = tiny.sparse(budget=400)
+    assert (sel[0, :, :236] >= 0).all()
+    assert np.abs(out - dense).max() <= 1e-5
+    check_output(x, out, x.prefix, x.window, None, dense=True)
+
+
+def test_budget_zero(tiny):
+    x = tiny.x
+    out, _ = tiny.sparse(budget=0)
+    check_output(x, out, x.prefix, x.window, np.full((1, 2, 0), -1, dtype=np.int32))
+
+
+def test_nan_sentinels_do_not_leak():
+    a = small(4, 8, 2, 128, [37, 600, 16, 1201], prefix=20, window=100, budget=5, fill="zero")
+    b = small(4, 8, 2, 128, [37, 600, 16, 1201], prefix=20, window=100, budget=5, fill="nan")
+    oa, sa = Dev(a).sparse()
+    ob, sb = Dev(b).sparse()
+    np.testing.assert_array_equal(sa, sb)
+    np.testing.assert_array_equal(oa, ob)
+    check_output(b, ob, 20, 100, sb)
+
+
+def test_layout_invariance():
+    a = small(3, 8, 2, 128, [900, 333, 2000], prefix=32, window=64, budget=6, layout="contiguous")
+    b = small(3, 8, 2, 128, [900, 333, 2000], prefix=32, window=64, budget=6, layout="shuffled")
+    oa, sa = Dev(a).sparse()
+    ob, sb = Dev(b).sparse()
+    np.testing.assert_array_equal(sa, sb)
+    assert np.abs(oa - ob).max() <= 1e-6
+
+
+@pytest.mark.parametrize("hq,hkv,D", [(8, 2, 128), (4, 4, 128), (6, 2, 128), (16, 2, 256),
+                                      (8, 8, 256)])
+def test_edge_lengths_and_groups(hq, hkv, D):
+    lens = [0, 1, 15, 16, 17, 33, 100, 257, 1999]
+    x = small(len(lens), hq, hkv, D, lens, seed=hq * 31 + D, fill="nan")
+    d = Dev(x)
+    meta_matches_oracle(d)
+    for P, Wn, K in [(0, 0, 3), (16, 32, 2), (5, 1, 0), (64, 256, 100), (0, 16, 1)]:
+        out, sel = d.sparse(P, Wn, K)
+        check_selection(x, sel, P, Wn, K)
+        check_output(x, out, P, Wn, sel)
+        assert (out[0] == 0).all()  # empty sequence
+    check_output(x, d.dense(), 0, 0, None, dense=True)
+
+
+def test_explicit_scale(tiny):
+    x = tiny.x
+    out, sel = tiny.sparse(scale=0.3)
+    want = oracle.attend(x.q, x.k_cache, x.v_cache, x.block_table, x.seq_lens, x.prefix,
+                         x.window, sel, scale=0.3)
+    assert np.abs(out - want).max() <= 2e-3
+
+
+def test_bad_block_table_entry_is_flagged_not_followed():
+    import sparse_long_context_max_b200 as slc
+    x = small(2, 8, 2, 128, [300, 300], prefix=16, window=32, budget=4)
+    d = Dev(x)
+    bt = d.bt.clone()
+    bt[1, 5] = x.k_cache.shape[0] + 1000  # outside the pool
+    bt[0, 7] = -3
+    slc.sparse_decode(d.q, d.cache, bt, d.sl, 16, 32, 4)
+    torch.cuda.synchronize()
+    st = slc.device_status()
+    assert st & 1  # bad page
+    assert slc.device_status() == 0  # cleared
+    bad_len = d.sl.clone()
+    bad_len[0] = 10 ** 6
+    slc.dense_decode(d.q, d.cache, d.bt, bad_len)
+    torch.cuda.synchronize()
+    assert slc.device_status() & 2
+
+
+# ------------------------------------------------------------------ workloads
+
+def test_ragged_workload_parity():
+    x = synth.make_inputs(W["ragged"], fill="nan")
+    d = Dev(x)
+    out, sel = d.sparse()
+    check_selection(x, sel, x.prefix, x.window, x.budget)
+    check_needles(x, sel)
+    check_output(x, out, x.prefix, x.window, sel)
+    # the two short sequences are covered whole: equal to dense attention
+    dense = d.dense()
+    assert np.abs(out[:2] - dense[:2]).max() <= 1e-5
+    xs = slice_batch(x, [0, 1, 5, 22])
+    check_output(xs, dense[[0, 1, 5, 22]], 0, 0, None, dense=True)
+
+
+def test_decode256k_parity():
+    x = synth.make_inputs(W["decode256k"])
+    d = Dev(x)
+    out, sel = d.sparse()
+    check_selection(x, sel, x.prefix, x.window, x.budget)
+    check_needles(x, sel)
+    check_output(x, out, x.prefix, x.window, sel)
+    dense = d.dense()
+    xs = slice_batch(x, [2])
+    check_output(xs, dense[[2]], 0, 0, None, dense=True)
+
+
+def test_decode64k_append_loop():
+    import sparse_long_context_max_b200 as slc
+    wl = W["decode64k"]
+    x = synth.make_inputs(wl)
+    d = Dev(x)
+    lens = x.seq_lens.clone()
+    check_at = {0, 1, 17, wl.steps - 1}
+    for step in range(wl.steps):
+        if step > 0:
+            q, kn, vn = synth.step_tokens(wl, step)
+            # append the new token, then decode with it in the context
+            slc.kv_append(d.cache, kn.cuda(), vn.cuda(), d.bt, lens.cuda())
+            for b in range(wl.batch):
+                L = int(lens[b])
+                phys = int(x.block_table[b, L // 16])
+                x.k_cache[phys, :, L % 16] = kn[b]
+                x.v_cache[phys, :, L % 16] = vn[b]
+            lens += 1
+            x.q = q
+            d.q = q.cuda()
+            x.seq_lens = lens.clone()
+            d.sl = lens.cuda()
+        if step in check_at:
+            out, sel = d.sparse()
+            check_selection(x, sel, x.prefix, x.window, x.budget)
+            if step == 0:
+                check_needles(x, sel)
+            check_output(x, out, x.prefix, x.window, sel)
+        else:
+            import sparse_long_context_max_b200 as s2
+            s2.sparse_decode(d.q, d.cache, d.bt, d.sl, x.prefix, x.window, x.budget)
+    torch.cuda.synchronize()
+    assert slc.device_status() == 0
+    incremental = d.cache.meta.clone()
+    slc.build_page_meta(d.cache, d.bt, d.sl)
+    used = x.block_table[:, : -(-int(lens.max()) // 16)].reshape(-1).long()
+    assert torch.equal(incremental[used.cuda()].float(), d.cache.meta[used.cuda()].float())
+
+
+def test_layers131k_sampled_layers():
+    wl = W["layers131k"]
+    plan = synth.layer_plan(wl)
+    dense_layer = [i for i, (_, _, dn) in enumerate(plan) if dn][0]
+    sparse_layers = [i for i, (_, _, dn) in enumerate(plan) if not dn][:2]
+    for layer in sparse_layers + [dense_layer]:
+        x = synth.make_inputs(wl, layer=layer)
+        d = Dev(x)
+        if plan[layer][2]:
+            out = d.dense()
+            check_output(slice_batch(x, [1]), out[[1]], 0, 0, None, dense=True)
+        else:
+            out, sel = d.sparse()
+            check_selection(x, sel, x.prefix, x.window, x.budget)
+            check_needles(x, sel)
+            check_output(x, out, x.prefix, x.window, sel)
+        del d, x
+        torch.cuda.empty_cache()
