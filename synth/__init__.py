@@ -250,8 +250,10 @@ def make_inputs(wl: Workload, layer: int = 0, fill: str = "zero",
         for job in jobs:
             work(job)
 
-    # planted needles: key = 4 x (mean of the group's query heads), at every
-    # kv head of the chosen token; placed well clear of prefix and window
+    # planted needles: at every kv head of the chosen token, the key points
+    # along the mean of that kv head's query heads, with 4x the typical key
+    # norm (keys are N(0,1) per dimension, so sqrt(D)); placed well clear of
+    # prefix and window
     nn = wl.needles if needles is None else needles
     needle_tokens = []
     G = Hq // Hkv
@@ -272,7 +274,8 @@ def make_inputs(wl: Workload, layer: int = 0, fill: str = "zero",
             for t in toks:
                 phys = int(bt[b, t // PAGE])
                 for h in range(Hkv):
-                    key = 4.0 * qf[b, h * G:(h + 1) * G, :].mean(dim=0)
+                    g_mean = qf[b, h * G:(h + 1) * G, :].mean(dim=0)
+                    key = 4.0 * math.sqrt(D) * g_mean / g_mean.norm()
                     kc[phys, h, t % PAGE, :] = key.to(torch.bfloat16)
         needle_tokens.append(toks)
 
