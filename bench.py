@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--no-also", action="store_true", help="skip the 256k/dense measurements")
     ap.add_argument("--reps", type=int, default=20, help="repetitions of each extra measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--profile", metavar="WORKLOAD", default=None,
+                    help="launch each kernel twice on WORKLOAD and exit (for ncu)")
     return ap.parse_args()
 
 
@@ -529,9 +531,36 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+def run_profile(name):
+    """Each entry point twice on one workload, nothing timed: the command
+    that ncu captures.  Launch order: build_meta, then twice (kv_append,
+    score, select, attend, merge), then dense (attend, merge)."""
+    import torch
+    import sparse_long_context_max_b200 as slc
+    w = Workload(name, extra_tokens=2)
+    x = w.x
+    B, hkv, D = x.q.shape[0], w.wl.hkv, w.wl.head_dim
+    pos = w.sl.clone()
+    for _ in range(2):
+        kn = torch.zeros((B, hkv, D), dtype=torch.bfloat16, device="cuda")
+        slc.kv_append(w.cache, kn, kn, w.bt, pos)
+        pos += 1
+        slc.sparse_decode(w.q, w.cache, w.bt, pos, x.prefix, x.window, x.budget, out=w.out,
+                          workspace=w.ws)
+    slc.dense_decode(w.q, w.cache, w.bt, pos, out=w.out, workspace=w.ws)
+    torch.cuda.synchronize()
+    st = slc.device_status()
+    print("profile run done: %s, status %d" % (name, st))
+    if st:
+        raise SystemExit(1)
+
+
 def main():
     args = parse()
     rank, world, local = rank_info()
+    if args.profile:
+        run_profile(args.profile)
+        return
     if args.impl == "reference":
         res = run_reference(args, rank, world)
         if res is not None:

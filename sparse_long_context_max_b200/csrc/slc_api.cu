@@ -84,7 +84,7 @@ WorkspaceLayout workspace_layout(int batch, int hq, int hkv, int head_dim, int m
     WorkspaceLayout w{};
     const size_t units = (size_t)batch * hkv;
     const size_t group = (size_t)(hq / hkv);
-    const size_t slots = units + kMaxAttendWarps;
+    const size_t slots = units + kMaxAttendChunks;
     size_t off = 0;
     w.scores = off;
     off = round_up(off + units * max_pages * sizeof(float), 256);

@@ -10,13 +10,15 @@
 //           (same article, section "The method: sliding window + prefix +
 //           query-aware pages, searched per layer")
 // The lists of all units are concatenated and cut into equal chunks, one per
-// warp of a persistent grid, so work is balanced by pages whatever the
+// CTA of a persistent grid, so work is balanced by pages whatever the
 // sequence lengths.  A chunk that spans unit boundaries yields one partial
 // (running max m, sum l, unnormalised accumulator) per unit piece, stored in
 // slot (unit + chunk), which is unique.  The merge kernel combines a unit's
 // partials: out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k.
 //
-// Per warp, pages stream through a private ring of shared-memory stages,
+// Within a CTA the warps take a piece's pages round-robin and combine their
+// partials in shared memory.  Per warp, pages stream through a private ring
+// of shared-memory stages,
 // each filled by two 1-D bulk copies (TMA engine: the K and V tiles of one
 // (page, kv head) are contiguous, 32*D bytes each) completing on an
 // mbarrier.  The group's query heads (G <= 8) and the 16 tokens of a page
@@ -88,12 +90,22 @@ __device__ __forceinline__ void issue_page(const AttendParams& p, const Ring& ri
     bulk_g2s(dst + TILE, static_cast<const __nv_bfloat16*>(p.v_cache) + off, TILE, bar);
 }
 
-// Process list positions [i0, i1) of unit u; write the partial to `slot`.
-// `it` counts ring uses of this warp (stage = it % STAGES).  Returns false
-// if a bounded wait gave up (the warp then stops).
+// Per-warp partial state: the running max of head r_ (log2 units), this
+// thread's share of the running sum, and the O^T accumulators of heads 2c,
+// 2c+1 over dims (D/8)*r_ .. (D/8)*r_ + D/8 - 1.
+template <int D>
+struct WarpState {
+    float m, l;
+    float acc[D / 16][4];
+};
+
+// Attend list positions i0, i0 + stride, ... < i1 of unit u with this warp's
+// ring.  `it` counts the warp's ring uses (stage = it % STAGES).  `ok` turns
+// false if a bounded wait gave up; the warp then drains its copies in flight
+// and skips all further work (it still reaches every CTA barrier).
 template <int D, int STAGES>
-__device__ bool attend_piece(const AttendParams& p, const Ring& ring, uint32_t& it, int u,
-                             int i0, int i1, long long slot) {
+__device__ void warp_attend(const AttendParams& p, const Ring& ring, uint32_t& it, bool& ok,
+                            int u, int i0, int i1, int stride, WarpState<D>& st) {
     constexpr int TILE_W = kPage * D / 2;  // 32-bit words per tile
     constexpr int ROW_W = D / 2;           // words per token row
     constexpr int KS = D / 16;             // k-steps of Q K^T, m-blocks of V^T P^T
@@ -101,10 +113,23 @@ __device__ bool attend_piece(const AttendParams& p, const Ring& ring, uint32_t& 
     const int r_ = lane >> 2, c_ = lane & 3;
     const int b = u / p.hkv, h = u % p.hkv;
     const int G = p.group;
+    st.m = -INFINITY;
+    st.l = 0.f;
+#pragma unroll
+    for (int i = 0; i < KS; ++i) st.acc[i][0] = st.acc[i][1] = st.acc[i][2] = st.acc[i][3] = 0.f;
+    const int npg = i1 > i0 ? (i1 - i0 + stride - 1) / stride : 0;
+    if (!ok || npg == 0) return;
     const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
     const PageRanges r = page_ranges(L, p.prefix, p.window);
     const int nsel = p.sparse ? min(p.budget, r.ws - r.np) : 0;
-    const int npg = i1 - i0;
+
+    __syncwarp();  // this warp's earlier reads of the ring are done
+    if (lane == 0) {
+        fence_proxy_async_smem();
+        for (int k = 0; k < STAGES && k < npg; ++k)
+            issue_page<D>(p, ring, (it + k) % STAGES, u, b, h, r, nsel, L, i0 + k * stride);
+    }
+    __syncwarp();
 
     // query fragments (rows >= G and rows 8..15 are zero)
     uint32_t qa[KS][2];
@@ -113,7 +138,7 @@ __device__ bool attend_piece(const AttendParams& p, const Ring& ring, uint32_t& 
             static_cast<const __nv_bfloat16*>(p.q) + ((long long)b * p.hq + h * G + r_) * D);
 #pragma unroll
         for (int m = 0; m < D / 32; ++m) {
-            const uint4 v = qrow[c_ + 4 * m];
+            const uint4 v = __ldg(qrow + c_ + 4 * m);
             qa[2 * m][0] = v.x;
             qa[2 * m][1] = v.y;
             qa[2 * m + 1][0] = v.z;
@@ -124,24 +149,10 @@ __device__ bool attend_piece(const AttendParams& p, const Ring& ring, uint32_t& 
         for (int k = 0; k < KS; ++k) qa[k][0] = qa[k][1] = 0u;
     }
 
-    __syncwarp();  // the previous piece's reads of the ring are done
-    if (lane == 0) {
-        fence_proxy_async_smem();
-        for (int k = 0; k < STAGES && k < npg; ++k)
-            issue_page<D>(p, ring, (it + k) % STAGES, u, b, h, r, nsel, L, i0 + k);
-    }
-    __syncwarp();
-
-    float m_run = -INFINITY, l_run = 0.f;
-    float acc[KS][4];
-#pragma unroll
-    for (int i = 0; i < KS; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-
     for (int k = 0; k < npg; ++k) {
         const uint32_t use = it + k;
         const int stage = use % STAGES;
         if (!mbar_wait_bounded(ring.bars + stage, (use / STAGES) & 1u, kWaitLimit)) {
-            // give up: record it, drain this warp's copies in flight, stop
             if (lane == 0) {
                 atomicOr(p.status, SLC_STATUS_WAIT_TIMEOUT);
                 for (int kk = k; kk < npg && kk < k + STAGES; ++kk) {
@@ -150,7 +161,8 @@ __device__ bool attend_piece(const AttendParams& p, const Ring& ring, uint32_t& 
                 }
             }
             __syncwarp();
-            return false;
+            ok = false;
+            return;
         }
         const uint32_t* Kw = reinterpret_cast<const uint32_t*>(ring.tiles) + stage * 2 * TILE_W;
         const uint32_t* Vw = Kw + TILE_W;
@@ -179,22 +191,22 @@ __device__ bool attend_piece(const AttendParams& p, const Ring& ring, uint32_t& 
         float pmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
         pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 1));
         pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 2));
-        const float m_new = fmaxf(m_run, pmax);
+        const float m_new = fmaxf(st.m, pmax);
         const float m_use = m_new == -INFINITY ? 0.f : m_new;
-        const float alpha = ex2(m_run - m_use);
+        const float alpha = ex2(st.m - m_use);
         float pr[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) pr[e] = ex2(x[e] - m_use);
-        l_run = l_run * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
-        m_run = m_new;
+        st.l = st.l * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
+        st.m = m_new;
         const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * c_);
         const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * c_ + 4);
 #pragma unroll
         for (int i = 0; i < KS; ++i) {
-            acc[i][0] *= a0;
-            acc[i][1] *= a1;
-            acc[i][2] *= a0;
-            acc[i][3] *= a1;
+            st.acc[i][0] *= a0;
+            st.acc[i][1] *= a1;
+            st.acc[i][2] *= a0;
+            st.acc[i][3] *= a1;
         }
         // P^T fragments (tokens 2c,2c+1 / 2c+8,2c+9 of head r_), hi + lo
         const uint32_t bh0 = pack_bf16x2(pr[0], pr[1]);
@@ -209,10 +221,10 @@ __device__ bool attend_piece(const AttendParams& p, const Ring& ring, uint32_t& 
         for (int tt = 0; tt < 4; ++tt) {
             const int tok = t0 + (tt & 1) + (tt >> 1) * 8;
             const uint32_t* vrow = Vw + tok * ROW_W + WPT * r_;
+            const bool live = tok < nv;  // zero slots past the length (may hold NaN)
 #pragma unroll
             for (int q4 = 0; q4 < WPT / 4; ++q4) {
                 const uint4 v = lds128(vrow + 4 * q4);
-                const bool live = tok < nv;  // zero slots past the length (may hold NaN)
                 vw[tt][4 * q4 + 0] = live ? v.x : 0u;
                 vw[tt][4 * q4 + 1] = live ? v.y : 0u;
                 vw[tt][4 * q4 + 2] = live ? v.z : 0u;
@@ -225,35 +237,19 @@ __device__ bool attend_piece(const AttendParams& p, const Ring& ring, uint32_t& 
             const uint32_t a1r = __byte_perm(vw[0][i], vw[1][i], 0x7632);
             const uint32_t a2r = __byte_perm(vw[2][i], vw[3][i], 0x5410);
             const uint32_t a3r = __byte_perm(vw[2][i], vw[3][i], 0x7632);
-            mma_bf16(acc[i], a0r, a1r, a2r, a3r, bh0, bh1);
-            mma_bf16(acc[i], a0r, a1r, a2r, a3r, bl0, bl1);
+            mma_bf16(st.acc[i], a0r, a1r, a2r, a3r, bh0, bh1);
+            mma_bf16(st.acc[i], a0r, a1r, a2r, a3r, bl0, bl1);
         }
         __syncwarp();
         if (lane == 0 && k + STAGES < npg) {
             fence_proxy_async_smem();
-            issue_page<D>(p, ring, stage, u, b, h, r, nsel, L, i0 + k + STAGES);
+            issue_page<D>(p, ring, stage, u, b, h, r, nsel, L, i0 + (k + STAGES) * stride);
         }
     }
     it += npg;
-
-    // partial: (m, l) of head r_, accumulators of heads 2c, 2c+1
-    float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 1);
-    l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
-    if (c_ == 0 && r_ < G) p.part_ml[slot * G + r_] = make_float2(m_run, l_tot);
-    constexpr int DPT = D / 8;
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        const int head = 2 * c_ + hh;
-        if (head < G) {
-            float4* dst =
-                reinterpret_cast<float4*>(p.part_acc + (slot * G + head) * D + DPT * r_);
-#pragma unroll
-            for (int i2 = 0; i2 < KS / 2; ++i2)
-                dst[i2] = make_float4(acc[2 * i2][hh], acc[2 * i2][2 + hh], acc[2 * i2 + 1][hh],
-                                      acc[2 * i2 + 1][2 + hh]);
-        }
-    }
-    return true;
+    // full sum of head r_ (the four threads of a quad hold parts of it)
+    st.l += __shfl_xor_sync(0xffffffffu, st.l, 1);
+    st.l += __shfl_xor_sync(0xffffffffu, st.l, 2);
 }
 
 __device__ __forceinline__ int list_len(const AttendParams& p, int b) {
@@ -263,33 +259,43 @@ __device__ __forceinline__ int list_len(const AttendParams& p, int b) {
     return r.np + min(p.budget, r.ws - r.np) + (r.n - r.ws);
 }
 
+// One CTA per chunk of the concatenated page lists.  For every unit piece
+// of the chunk, the CTA's warps take its pages round-robin, then combine
+// their partials in shared memory (reusing their rings) into one partial,
+// stored in slot (unit + chunk).
 template <int D, int NW, int STAGES>
 __global__ void __launch_bounds__(NW * 32) attend_kernel(AttendParams p) {
     constexpr int TILE = kPage * D * 2;
+    constexpr int RING = STAGES * 2 * TILE;
+    constexpr int KS = D / 16;
+    constexpr int DPT = D / 8;
+    static_assert(RING >= (kMaxGroup * D + 2 * kMaxGroup) * 4, "ring holds a warp partial");
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r_ = lane >> 2, c_ = lane & 3;
     Ring ring;
-    ring.tiles = smem + warp * STAGES * 2 * TILE;
-    ring.bars = reinterpret_cast<uint64_t*>(smem + NW * STAGES * 2 * TILE) + warp * STAGES;
-    ring.nvalid = reinterpret_cast<int*>(smem + NW * STAGES * 2 * TILE + NW * STAGES * 8) +
-                  warp * STAGES;
+    ring.tiles = smem + warp * RING;
+    ring.bars = reinterpret_cast<uint64_t*>(smem + NW * RING) + warp * STAGES;
+    ring.nvalid = reinterpret_cast<int*>(smem + NW * RING + NW * STAGES * 8) + warp * STAGES;
     if (lane == 0) {
         for (int s = 0; s < STAGES; ++s) mbar_init(ring.bars + s, 1);
         fence_mbar_init();
     }
     __syncwarp();
 
-    const int gw = blockIdx.x * NW + warp;
     auto len_of = [&](int b) { return list_len(p, b); };
     const long long total = total_units(p.batch, p.hkv, len_of);
-    const long long cpp = (total + p.total_warps - 1) / p.total_warps;
-    long long s = (long long)gw * cpp;
+    const long long cpp = (total + gridDim.x - 1) / gridDim.x;
+    long long s = (long long)blockIdx.x * cpp;
     const long long e = min(total, s + cpp);
-    if (s >= e) return;
+    if (s >= e) return;  // uniform across the CTA
     int u;
     long long ustart;
     locate_unit(s, p.batch, p.hkv, len_of, &u, &ustart);
     uint32_t it = 0;
+    bool ok = true;
+    const int G = p.group;
+    WarpState<D> st;
     while (s < e) {
         const int len = list_len(p, u / p.hkv);
         if (len == 0) {
@@ -298,63 +304,140 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttendParams p) {
         }
         const int i0 = (int)(s - ustart);
         const int i1 = (int)(min(e, ustart + len) - ustart);
-        if (!attend_piece<D, STAGES>(p, ring, it, u, i0, i1, (long long)u + gw)) return;
+        warp_attend<D, STAGES>(p, ring, it, ok, u, i0 + warp, i1, NW, st);
+
+        // combine the NW warp partials through shared memory
+        __syncthreads();  // every warp is done with its ring
+        float* wacc = reinterpret_cast<float*>(smem + warp * RING);  // [G][D]
+        float2* wml = reinterpret_cast<float2*>(wacc + kMaxGroup * D);  // [G]
+        if (c_ == 0 && r_ < G) wml[r_] = make_float2(st.m, st.l);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int head = 2 * c_ + hh;
+            if (head < G) {
+                float4* dst = reinterpret_cast<float4*>(wacc + head * D + DPT * r_);
+#pragma unroll
+                for (int i2 = 0; i2 < KS / 2; ++i2)
+                    dst[i2] = make_float4(st.acc[2 * i2][hh], st.acc[2 * i2][2 + hh],
+                                          st.acc[2 * i2 + 1][hh], st.acc[2 * i2 + 1][2 + hh]);
+            }
+        }
+        __syncthreads();
+        const long long slot = (long long)u + blockIdx.x;
+        for (int item = threadIdx.x; item < G * (D / 4); item += NW * 32) {
+            const int g = item / (D / 4), d4 = item % (D / 4);
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float2 ml = reinterpret_cast<const float2*>(
+                    reinterpret_cast<const float*>(smem + w * RING) + kMaxGroup * D)[g];
+                M = fmaxf(M, ml.x);
+            }
+            const float Mu = M == -INFINITY ? 0.f : M;
+            float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+            float den = 0.f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float* wa = reinterpret_cast<const float*>(smem + w * RING);
+                const float2 ml = reinterpret_cast<const float2*>(wa + kMaxGroup * D)[g];
+                const float wt = ex2(ml.x - Mu);
+                const float4 a = reinterpret_cast<const float4*>(wa + g * D)[d4];
+                num.x = fmaf(wt, a.x, num.x);
+                num.y = fmaf(wt, a.y, num.y);
+                num.z = fmaf(wt, a.z, num.z);
+                num.w = fmaf(wt, a.w, num.w);
+                den = fmaf(wt, ml.y, den);
+            }
+            reinterpret_cast<float4*>(p.part_acc + (slot * G + g) * D)[d4] = num;
+            if (d4 == 0) p.part_ml[slot * G + g] = make_float2(M, den);
+        }
+        __syncthreads();  // the rings are reused by the next piece
         s = ustart + len;
         ustart = s;
         ++u;
     }
 }
 
-// One CTA per unit: combine the unit's partials (slots unit + chunk).
+// Merge of the CTA partials of one (unit, query head): slots unit + chunk
+// for the chunks that cover the unit.  The block's threads split into
+// MERGE_GROUPS slot groups x D/4 dimension quads; groups combine in shared
+// memory.
+constexpr int kMergeGroups = 4;
+
 template <int D>
-__global__ void __launch_bounds__(256) merge_kernel(AttendParams p) {
-    const int u = blockIdx.x;
+__global__ void __launch_bounds__(kMergeGroups * D / 4) merge_kernel(AttendParams p) {
+    constexpr int V4 = D / 4;
+    const int u = blockIdx.x, g = blockIdx.y;
     const int b = u / p.hkv, h = u % p.hkv;
     const int G = p.group;
-    __shared__ long long sh_off;
-    __shared__ long long sh_total;
-    if (threadIdx.x < 32) {
-        // offset of unit u in the concatenated lists, and the total
+    const int tid = threadIdx.x;
+    const int grp = tid / V4, d4 = tid % V4;
+    __shared__ long long sh_off, sh_total;
+    __shared__ float sh_m[kMergeGroups];
+    __shared__ float4 sh_num[kMergeGroups][V4];
+    __shared__ float sh_den[kMergeGroups];
+    if (tid < 32) {
         auto len_of = [&](int bb) { return list_len(p, bb); };
         const long long total = total_units(p.batch, p.hkv, len_of);
         long long base = 0;
         for (int b0 = 0; b0 < b; b0 += 32) {
-            const int bb = b0 + threadIdx.x;
+            const int bb = b0 + tid;
             long long c = bb < b ? (long long)list_len(p, bb) * p.hkv : 0;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
             base += c;
         }
-        if (threadIdx.x == 0) {
+        if (tid == 0) {
             sh_off = base + (long long)h * list_len(p, b);
             sh_total = total;
         }
     }
     __syncthreads();
     const int len = list_len(p, b);
-    const long long cpp = (sh_total + p.total_warps - 1) / p.total_warps;
-    const long long k0 = len > 0 ? sh_off / cpp : 0;
-    const long long k1 = len > 0 ? (sh_off + len - 1) / cpp : -1;
-    constexpr int V4 = D / 4;
-    for (int item = threadIdx.x; item < G * V4; item += blockDim.x) {
-        const int g = item / V4, d4 = item % V4;
-        float M = -INFINITY;
-        for (long long k = k0; k <= k1; ++k) M = fmaxf(M, p.part_ml[(u + k) * G + g].x);
-        const float Mu = M == -INFINITY ? 0.f : M;
-        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-        float den = 0.f;
-        for (long long k = k0; k <= k1; ++k) {
-            const float2 ml = p.part_ml[(u + k) * G + g];
-            const float w = ex2(ml.x - Mu);
-            const float4 a = reinterpret_cast<const float4*>(p.part_acc + ((u + k) * G + g) * D)[d4];
-            num.x = fmaf(w, a.x, num.x);
-            num.y = fmaf(w, a.y, num.y);
-            num.z = fmaf(w, a.z, num.z);
-            num.w = fmaf(w, a.w, num.w);
-            den = fmaf(w, ml.y, den);
+    float* outp = p.out + ((long long)b * p.hq + h * G + g) * D;
+    if (len == 0) {
+        if (grp == 0) reinterpret_cast<float4*>(outp)[d4] = make_float4(0.f, 0.f, 0.f, 0.f);
+        return;
+    }
+    const long long cpp = (sh_total + p.num_chunks - 1) / p.num_chunks;
+    const long long k0 = sh_off / cpp, k1 = (sh_off + len - 1) / cpp;
+    // 1) the unit's maximum
+    float M = -INFINITY;
+    for (long long k = k0 + grp; k <= k1; k += kMergeGroups)
+        M = fmaxf(M, __ldg(&p.part_ml[(u + k) * G + g].x));
+    if (d4 == 0) sh_m[grp] = M;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kMergeGroups; ++i) M = fmaxf(M, sh_m[i]);
+    const float Mu = M == -INFINITY ? 0.f : M;
+    // 2) weighted sums; slots of a group are independent loads
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    float den = 0.f;
+#pragma unroll 4
+    for (long long k = k0 + grp; k <= k1; k += kMergeGroups) {
+        const float2 ml = __ldg(&p.part_ml[(u + k) * G + g]);
+        const float4 a = __ldg(reinterpret_cast<const float4*>(p.part_acc + ((u + k) * G + g) * D) + d4);
+        const float w = ex2(ml.x - Mu);
+        num.x = fmaf(w, a.x, num.x);
+        num.y = fmaf(w, a.y, num.y);
+        num.z = fmaf(w, a.z, num.z);
+        num.w = fmaf(w, a.w, num.w);
+        den = fmaf(w, ml.y, den);
+    }
+    sh_num[grp][d4] = num;
+    if (d4 == 0) sh_den[grp] = den;
+    __syncthreads();
+    if (grp == 0) {
+        for (int i = 1; i < kMergeGroups; ++i) {
+            const float4 o = sh_num[i][d4];
+            num.x += o.x;
+            num.y += o.y;
+            num.z += o.z;
+            num.w += o.w;
+            den += sh_den[i];
         }
         const float inv = den > 0.f ? 1.f / den : 0.f;
-        reinterpret_cast<float4*>(p.out + ((long long)b * p.hq + h * G + g) * D)[d4] =
+        reinterpret_cast<float4*>(outp)[d4] =
             make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
     }
 }
@@ -378,12 +461,12 @@ cudaError_t run(AttendParams p, int num_sms, cudaStream_t stream, int* launched)
         if (occ < 1) occ = 1;
     }
     int blocks = num_sms * occ;
-    if (blocks * NW > kMaxAttendWarps) blocks = kMaxAttendWarps / NW;
-    p.total_warps = blocks * NW;
+    if (blocks > kMaxAttendChunks) blocks = kMaxAttendChunks;
+    p.num_chunks = blocks;  // chunk count (one chunk per CTA)
     attend_kernel<D, NW, STAGES><<<blocks, NW * 32, smem, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    merge_kernel<D><<<p.batch * p.hkv, 256, 0, stream>>>(p);
+    merge_kernel<D><<<dim3(p.batch * p.hkv, p.group), kMergeGroups * D / 4, 0, stream>>>(p);
     if (launched) *launched += 2;
     return cudaGetLastError();
 }

@@ -8,9 +8,9 @@
 
 namespace slc {
 
-// Upper bound on the number of attention warps of one launch; sizes the
-// split-partial workspace (slot = unit + warp chunk index).
-constexpr int kMaxAttendWarps = 4096;
+// Upper bound on the number of attention CTAs (chunks) of one launch; sizes
+// the split-partial workspace (slot = unit + chunk index).
+constexpr int kMaxAttendChunks = 1024;
 
 struct KvAppendParams {
     const void* k_new;
@@ -65,7 +65,7 @@ struct AttendParams {
     int batch, hq, hkv, group, max_pages, num_pages;
     int sparse, prefix, window, budget;
     float scale_log2;  // softmax scale * log2(e)
-    int total_warps;   // warps of the attention launch (chunk count)
+    int num_chunks;    // chunks of the attention launch (one per CTA)
 };
 
 // Workspace carve-up shared by the API and the size query.

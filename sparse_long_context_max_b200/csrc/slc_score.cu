@@ -87,15 +87,24 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreParams p) {
                 const int d0 = 8 * (chunk % CPR);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) w[m][e] = 0.f;
-                for (int gq = 0; gq < p.group; ++gq) {
-                    const uint4 qv = *reinterpret_cast<const uint4*>(
-                        static_cast<const __nv_bfloat16*>(p.q) +
-                        ((long long)b * p.hq + h * p.group + gq) * D + d0);
-                    const float qf[8] = {bf16_lo(qv.x), bf16_hi(qv.x), bf16_lo(qv.y), bf16_hi(qv.y),
-                                         bf16_lo(qv.z), bf16_hi(qv.z), bf16_lo(qv.w), bf16_hi(qv.w)};
+                // all group rows are loaded before any is used (one round trip)
+                uint4 qv[kMaxGroup];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        w[m][e] += is_max ? fmaxf(qf[e], 0.f) : fminf(qf[e], 0.f);
+                for (int gq = 0; gq < kMaxGroup; ++gq)
+                    if (gq < p.group)
+                        qv[gq] = __ldg(reinterpret_cast<const uint4*>(
+                            static_cast<const __nv_bfloat16*>(p.q) +
+                            ((long long)b * p.hq + h * p.group + gq) * D + d0));
+#pragma unroll
+                for (int gq = 0; gq < kMaxGroup; ++gq) {
+                    if (gq < p.group) {
+                        const float qf[8] = {bf16_lo(qv[gq].x), bf16_hi(qv[gq].x), bf16_lo(qv[gq].y),
+                                             bf16_hi(qv[gq].y), bf16_lo(qv[gq].z), bf16_hi(qv[gq].z),
+                                             bf16_lo(qv[gq].w), bf16_hi(qv[gq].w)};
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            w[m][e] += is_max ? fmaxf(qf[e], 0.f) : fminf(qf[e], 0.f);
+                    }
                 }
             }
         }
@@ -111,22 +120,25 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreParams p) {
 
         const uint4* meta = static_cast<const uint4*>(p.meta);
         float acc[32];
+        // every load of a phase is issued before the first is used: PH pages
+        // x CPL chunks = 32 x 16 bytes in flight per lane
+        constexpr int PH = 32 / CPL;
 #pragma unroll
-        for (int grp = 0; grp < 4; ++grp) {
-            uint4 v[8][CPL];
+        for (int ph0 = 0; ph0 < 32; ph0 += PH) {
+            uint4 v[PH][CPL];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int ph = __shfl_sync(0xffffffffu, phys, grp * 8 + i);
-                const uint4* base = meta + ((long long)ph * p.hkv + h) * (2 * CPR);
+            for (int i = 0; i < PH; ++i) {
+                const int pg = __shfl_sync(0xffffffffu, phys, ph0 + i);
+                const uint4* base = meta + ((long long)pg * p.hkv + h) * (2 * CPR);
 #pragma unroll
                 for (int m = 0; m < CPL; ++m) v[i][m] = __ldg(base + lane + 32 * m);
             }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < PH; ++i) {
                 float s = 0.f;
 #pragma unroll
                 for (int m = 0; m < CPL; ++m) s += dot8(w[m], v[i][m]);
-                acc[grp * 8 + i] = s;
+                acc[ph0 + i] = s;
             }
         }
         // transposed butterfly: after level `lvl`, a lane keeps the half of

@@ -54,9 +54,18 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectParams p) {
 
     // coalesced load, transposed through padded shared memory
     const float* s = p.scores + (long long)u * p.max_pages + r.np;
-    for (int i = tid; i < kThreads * KPT; i += kThreads) {
-        const uint32_t key = i < ncand ? order_key(s[i]) : 0u;
-        keys_smem[(i / KPT) * (KPT + 1) + (i % KPT)] = key;
+    {
+        float v[KPT];  // all loads in flight before the first store
+#pragma unroll
+        for (int k = 0; k < KPT; ++k) {
+            const int i = tid + k * kThreads;
+            v[k] = i < ncand ? __ldg(s + i) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < KPT; ++k) {
+            const int i = tid + k * kThreads;
+            keys_smem[(i / KPT) * (KPT + 1) + (i % KPT)] = i < ncand ? order_key(v[k]) : 0u;
+        }
     }
     __syncthreads();
     uint32_t key[KPT];
