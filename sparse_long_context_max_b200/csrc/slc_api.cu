@@ -29,9 +29,9 @@ DeviceInfo g_devices[kMaxDevices];
 std::mutex g_mutex;
 thread_local char g_cuda_error[256];
 
-int note_cuda(cudaError_t e) {
-    snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),
-             cudaGetErrorString(e));
+int note_cuda(cudaError_t e, const char* where = "") {
+    snprintf(g_cuda_error, sizeof g_cuda_error, "%s%s%s: %s", where, *where ? ": " : "",
+             cudaGetErrorName(e), cudaGetErrorString(e));
     return SLC_ERR_CUDA;
 }
 
@@ -88,6 +88,8 @@ WorkspaceLayout workspace_layout(int batch, int hq, int hkv, int head_dim, int m
     size_t off = 0;
     w.scores = off;
     off = round_up(off + units * max_pages * sizeof(float), 256);
+    w.tile_max = off;
+    off = round_up(off + units * tile_stride_of(max_pages) * sizeof(float), 256);
     w.selected = off;
     off = round_up(off + units * (size_t)(budget > 0 ? budget : 1) * sizeof(int32_t), 256);
     w.part_acc = off;
@@ -176,9 +178,10 @@ int slc_score_pages(const void* q, const slc_cache_t* cache, const int32_t* bloc
     if (!q || !block_table || !seq_lens || !scores || !aligned16(q)) return SLC_ERR_INVALID_ARG;
     DeviceInfo* dev;
     if ((rc = device_info(&dev))) return rc;
-    ScoreParams p{q,     cache->meta, block_table, seq_lens, scores, dev->status, batch,
+    ScoreParams p{q,           cache->meta, block_table, seq_lens,
+                  scores,      nullptr,     dev->status, batch,
                   num_q_heads, cache->num_kv_heads, num_q_heads / cache->num_kv_heads,
-                  max_pages_per_seq, cache->num_pages, prefix, window};
+                  max_pages_per_seq, cache->num_pages, prefix, window, 0};
     cudaError_t e = launch_score(p, cache->head_dim, dev->num_sms, stream);
     return e == cudaSuccess ? SLC_OK : note_cuda(e);
 }
@@ -195,8 +198,8 @@ int slc_select_pages(const float* scores, int32_t num_kv_heads, int32_t max_page
     DeviceInfo* dev;
     int rc;
     if ((rc = device_info(&dev))) return rc;
-    SelectParams p{scores, seq_lens, selected, dev->status, batch, num_kv_heads,
-                   max_pages_per_seq, prefix, window, budget};
+    SelectParams p{scores, nullptr, seq_lens, selected, dev->status, batch, num_kv_heads,
+                   max_pages_per_seq, prefix, window, budget, 0};
     cudaError_t e = launch_select(p, stream);
     return e == cudaSuccess ? SLC_OK : note_cuda(e);
 }
@@ -233,16 +236,18 @@ static int decode(int mode, const void* q, const slc_cache_t* cache,
     cudaError_t e = cudaSuccess;
     if (mode == 1 && budget > 0) {
         float* scores = reinterpret_cast<float*>(ws + w.scores);
+        float* tmax = reinterpret_cast<float*>(ws + w.tile_max);
+        const int ts = tile_stride_of(max_pages_per_seq);
         ScoreParams sp{q,           cache->meta, block_table, seq_lens,
-                       scores,      dev->status, batch,       num_q_heads,
-                       hkv,         num_q_heads / hkv,        max_pages_per_seq,
-                       cache->num_pages, prefix,  window};
+                       scores,      tmax,        dev->status, batch,
+                       num_q_heads, hkv,         num_q_heads / hkv, max_pages_per_seq,
+                       cache->num_pages, prefix, window, ts};
         e = launch_score(sp, D, dev->num_sms, stream);
-        if (e != cudaSuccess) return note_cuda(e);
-        SelectParams lp{scores, seq_lens, sel, dev->status, batch, hkv, max_pages_per_seq,
-                        prefix, window, budget};
+        if (e != cudaSuccess) return note_cuda(e, "score_pages");
+        SelectParams lp{scores, tmax,   seq_lens, sel,    dev->status, batch, hkv,
+                        max_pages_per_seq, prefix, window, budget, ts};
         e = launch_select(lp, stream);
-        if (e != cudaSuccess) return note_cuda(e);
+        if (e != cudaSuccess) return note_cuda(e, "select_pages");
     }
     AttendParams ap{};
     ap.q = q;
@@ -267,7 +272,7 @@ static int decode(int mode, const void* q, const slc_cache_t* cache,
     ap.budget = sparse ? budget : 0;
     ap.scale_log2 = scale * 1.4426950408889634f;
     e = launch_attend(ap, D, dev->num_sms, stream, nullptr);
-    return e == cudaSuccess ? SLC_OK : note_cuda(e);
+    return e == cudaSuccess ? SLC_OK : note_cuda(e, "attend/merge");
 }
 
 int slc_sparse_decode(const void* q, const slc_cache_t* cache, const int32_t* block_table,

@@ -46,41 +46,55 @@ struct Ring {
     int* nvalid;     // STAGES
 };
 
-// Logical page of list position i of a unit (and whether it is sane).
-__device__ __forceinline__ int list_page(const AttendParams& p, int u, const PageRanges& r,
-                                         int nsel, int i, bool* ok) {
-    *ok = true;
-    if (!p.sparse || i < r.np) return i;
-    if (i < r.np + nsel) {
-        const int j = p.selected[(long long)u * p.budget + (i - r.np)];
-        if (j < r.np || j >= r.ws) {
-            *ok = false;
-            return 0;
-        }
-        return j;
-    }
-    return r.ws + (i - r.np - nsel);
+// A unit's list: dense = pages 0..n-1; sparse = prefix pages, window pages,
+// then the selected pages (forced pages first, so they need no selection).
+__device__ __forceinline__ bool list_is_selected(const AttendParams& p, const PageRanges& r,
+                                                 int i) {
+    return p.sparse && i >= r.np + (r.n - r.ws);
 }
 
-template <int D>
-__device__ __forceinline__ void issue_page(const AttendParams& p, const Ring& ring, int stage,
-                                           int u, int b, int h, const PageRanges& r, int nsel,
-                                           int L, int i) {
-    constexpr uint32_t TILE = kPage * D * 2;
+// Logical page of list position i of a unit (and whether it is sane).
+__device__ __forceinline__ int list_page(const AttendParams& p, int u, const PageRanges& r,
+                                         int i, bool* ok) {
+    *ok = true;
+    if (!p.sparse || i < r.np) return i;
+    const int nwin = r.n - r.ws;
+    if (i < r.np + nwin) return r.ws + (i - r.np);
+    const int j = p.selected[(long long)u * p.budget + (i - r.np - nwin)];
+    if (j < r.np || j >= r.ws) {
+        *ok = false;
+        return 0;
+    }
+    return j;
+}
+
+// Physical page and valid-token count of list position i of unit u;
+// (0, 0) for an entry that fails its range check (flagged, then skipped).
+__device__ __forceinline__ void resolve_page(const AttendParams& p, int u, int b,
+                                             const PageRanges& r, int L, int i, int* phys,
+                                             int* nv) {
     bool ok;
-    const int j = list_page(p, u, r, nsel, i, &ok);
-    int phys = 0, nv = 0;
+    const int j = list_page(p, u, r, i, &ok);
+    *phys = 0;
+    *nv = 0;
     if (!ok) {
         atomicOr(p.status, SLC_STATUS_BAD_SELECTION);
-    } else {
-        phys = p.block_table[(long long)b * p.max_pages + j];
-        if (phys < 0 || phys >= p.num_pages) {
-            atomicOr(p.status, SLC_STATUS_BAD_PAGE);
-            phys = 0;
-        } else {
-            nv = min(kPage, L - j * kPage);
-        }
+        return;
     }
+    const int ph = p.block_table[(long long)b * p.max_pages + j];
+    if (ph < 0 || ph >= p.num_pages) {
+        atomicOr(p.status, SLC_STATUS_BAD_PAGE);
+        return;
+    }
+    *phys = ph;
+    *nv = min(kPage, L - j * kPage);
+}
+
+// Lane 0: bulk-copy the K and V tiles of (phys, h) into ring stage `stage`.
+template <int D>
+__device__ __forceinline__ void issue_kv(const AttendParams& p, const Ring& ring, int stage,
+                                         int h, int phys, int nv) {
+    constexpr uint32_t TILE = kPage * D * 2;
     ring.nvalid[stage] = nv;
     uint64_t* bar = ring.bars + stage;
     mbar_arrive_expect_tx(bar, 2 * TILE);
@@ -121,13 +135,24 @@ __device__ void warp_attend(const AttendParams& p, const Ring& ring, uint32_t& i
     if (!ok || npg == 0) return;
     const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
     const PageRanges r = page_ranges(L, p.prefix, p.window);
-    const int nsel = p.sparse ? min(p.budget, r.ws - r.np) : 0;
 
+    // page ids of this warp's pages, 32 at a time: lane t holds page k0 + t.
+    // Selected pages come from the preceding (selection) kernel: wait for
+    // it only when a batch holds one.
+    int id_phys = 0, id_nv = 0;
+    auto load_ids = [&](int k0) {
+        const int k = k0 + lane;
+        const bool sel = k < npg && list_is_selected(p, r, i0 + k * stride);
+        if (__any_sync(0xffffffffu, sel)) grid_dep_wait();
+        if (k < npg) resolve_page(p, u, b, r, L, i0 + k * stride, &id_phys, &id_nv);
+    };
+    load_ids(0);
     __syncwarp();  // this warp's earlier reads of the ring are done
-    if (lane == 0) {
-        fence_proxy_async_smem();
-        for (int k = 0; k < STAGES && k < npg; ++k)
-            issue_page<D>(p, ring, (it + k) % STAGES, u, b, h, r, nsel, L, i0 + k * stride);
+    fence_proxy_async_smem();
+    for (int k = 0; k < STAGES && k < npg; ++k) {
+        const int ph = __shfl_sync(0xffffffffu, id_phys, k);
+        const int nv = __shfl_sync(0xffffffffu, id_nv, k);
+        if (lane == 0) issue_kv<D>(p, ring, (it + k) % STAGES, h, ph, nv);
     }
     __syncwarp();
 
@@ -199,14 +224,16 @@ __device__ void warp_attend(const AttendParams& p, const Ring& ring, uint32_t& i
         for (int e = 0; e < 4; ++e) pr[e] = ex2(x[e] - m_use);
         st.l = st.l * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
         st.m = m_new;
-        const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * c_);
-        const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * c_ + 4);
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {  // some head's maximum moved
+            const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * c_);
+            const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * c_ + 4);
 #pragma unroll
-        for (int i = 0; i < KS; ++i) {
-            st.acc[i][0] *= a0;
-            st.acc[i][1] *= a1;
-            st.acc[i][2] *= a0;
-            st.acc[i][3] *= a1;
+            for (int i = 0; i < KS; ++i) {
+                st.acc[i][0] *= a0;
+                st.acc[i][1] *= a1;
+                st.acc[i][2] *= a0;
+                st.acc[i][3] *= a1;
+            }
         }
         // P^T fragments (tokens 2c,2c+1 / 2c+8,2c+9 of head r_), hi + lo
         const uint32_t bh0 = pack_bf16x2(pr[0], pr[1]);
@@ -221,14 +248,21 @@ __device__ void warp_attend(const AttendParams& p, const Ring& ring, uint32_t& i
         for (int tt = 0; tt < 4; ++tt) {
             const int tok = t0 + (tt & 1) + (tt >> 1) * 8;
             const uint32_t* vrow = Vw + tok * ROW_W + WPT * r_;
-            const bool live = tok < nv;  // zero slots past the length (may hold NaN)
 #pragma unroll
             for (int q4 = 0; q4 < WPT / 4; ++q4) {
                 const uint4 v = lds128(vrow + 4 * q4);
-                vw[tt][4 * q4 + 0] = live ? v.x : 0u;
-                vw[tt][4 * q4 + 1] = live ? v.y : 0u;
-                vw[tt][4 * q4 + 2] = live ? v.z : 0u;
-                vw[tt][4 * q4 + 3] = live ? v.w : 0u;
+                vw[tt][4 * q4 + 0] = v.x;
+                vw[tt][4 * q4 + 1] = v.y;
+                vw[tt][4 * q4 + 2] = v.z;
+                vw[tt][4 * q4 + 3] = v.w;
+            }
+        }
+        if (nv < kPage) {  // partial page: zero slots past the length (may hold NaN)
+#pragma unroll
+            for (int tt = 0; tt < 4; ++tt) {
+                const bool live = t0 + (tt & 1) + (tt >> 1) * 8 < nv;
+#pragma unroll
+                for (int i = 0; i < WPT; ++i) vw[tt][i] = live ? vw[tt][i] : 0u;
             }
         }
 #pragma unroll
@@ -241,9 +275,15 @@ __device__ void warp_attend(const AttendParams& p, const Ring& ring, uint32_t& i
             mma_bf16(st.acc[i], a0r, a1r, a2r, a3r, bl0, bl1);
         }
         __syncwarp();
-        if (lane == 0 && k + STAGES < npg) {
-            fence_proxy_async_smem();
-            issue_page<D>(p, ring, stage, u, b, h, r, nsel, L, i0 + (k + STAGES) * stride);
+        const int kn = k + STAGES;
+        if (kn < npg) {  // refill this stage (warp-uniform branch)
+            if ((kn & 31) == 0) load_ids(kn);
+            const int ph = __shfl_sync(0xffffffffu, id_phys, kn & 31);
+            const int nv = __shfl_sync(0xffffffffu, id_nv, kn & 31);
+            if (lane == 0) {
+                fence_proxy_async_smem();
+                issue_kv<D>(p, ring, stage, h, ph, nv);
+            }
         }
     }
     it += npg;
@@ -282,6 +322,7 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttendParams p) {
         fence_mbar_init();
     }
     __syncwarp();
+    grid_dep_launch();  // the merge may start; it waits before reading partials
 
     auto len_of = [&](int b) { return list_len(p, b); };
     const long long total = total_units(p.batch, p.hkv, len_of);
@@ -306,7 +347,9 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttendParams p) {
         const int i1 = (int)(min(e, ustart + len) - ustart);
         warp_attend<D, STAGES>(p, ring, it, ok, u, i0 + warp, i1, NW, st);
 
-        // combine the NW warp partials through shared memory
+        // combine the NW warp partials through shared memory; global writes
+        // only after the preceding kernel has completed
+        grid_dep_wait();
         __syncthreads();  // every warp is done with its ring
         float* wacc = reinterpret_cast<float*>(smem + warp * RING);  // [G][D]
         float2* wml = reinterpret_cast<float2*>(wacc + kMaxGroup * D);  // [G]
@@ -396,28 +439,32 @@ __global__ void __launch_bounds__(kMergeGroups * D / 4) merge_kernel(AttendParam
     const int len = list_len(p, b);
     float* outp = p.out + ((long long)b * p.hq + h * G + g) * D;
     if (len == 0) {
+        grid_dep_wait();
         if (grp == 0) reinterpret_cast<float4*>(outp)[d4] = make_float4(0.f, 0.f, 0.f, 0.f);
         return;
     }
     const long long cpp = (sh_total + p.num_chunks - 1) / p.num_chunks;
     const long long k0 = sh_off / cpp, k1 = (sh_off + len - 1) / cpp;
-    // 1) the unit's maximum
-    float M = -INFINITY;
-    for (long long k = k0 + grp; k <= k1; k += kMergeGroups)
-        M = fmaxf(M, __ldg(&p.part_ml[(u + k) * G + g].x));
-    if (d4 == 0) sh_m[grp] = M;
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < kMergeGroups; ++i) M = fmaxf(M, sh_m[i]);
-    const float Mu = M == -INFINITY ? 0.f : M;
-    // 2) weighted sums; slots of a group are independent loads
+    grid_dep_wait();  // the partials come from the attention kernel
+    // one pass per slot group with online rescaling; slots of a group are
+    // independent loads
+    float M = -INFINITY, den = 0.f;
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-    float den = 0.f;
 #pragma unroll 4
     for (long long k = k0 + grp; k <= k1; k += kMergeGroups) {
         const float2 ml = __ldg(&p.part_ml[(u + k) * G + g]);
-        const float4 a = __ldg(reinterpret_cast<const float4*>(p.part_acc + ((u + k) * G + g) * D) + d4);
-        const float w = ex2(ml.x - Mu);
+        const float4 a =
+            __ldg(reinterpret_cast<const float4*>(p.part_acc + ((u + k) * G + g) * D) + d4);
+        if (ml.x > M) {  // new maximum: rescale what was summed so far
+            const float c = ex2(M - ml.x);
+            num.x *= c;
+            num.y *= c;
+            num.z *= c;
+            num.w *= c;
+            den *= c;
+            M = ml.x;
+        }
+        const float w = ml.x == -INFINITY ? 0.f : ex2(ml.x - M);  // empty partial
         num.x = fmaf(w, a.x, num.x);
         num.y = fmaf(w, a.y, num.y);
         num.z = fmaf(w, a.z, num.z);
@@ -425,20 +472,31 @@ __global__ void __launch_bounds__(kMergeGroups * D / 4) merge_kernel(AttendParam
         den = fmaf(w, ml.y, den);
     }
     sh_num[grp][d4] = num;
-    if (d4 == 0) sh_den[grp] = den;
+    if (d4 == 0) {
+        sh_den[grp] = den;
+        sh_m[grp] = M;
+    }
     __syncthreads();
     if (grp == 0) {
-        for (int i = 1; i < kMergeGroups; ++i) {
+        float Mt = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kMergeGroups; ++i) Mt = fmaxf(Mt, sh_m[i]);
+        const float Mu = Mt == -INFINITY ? 0.f : Mt;
+        float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
+        float dt = 0.f;
+#pragma unroll
+        for (int i = 0; i < kMergeGroups; ++i) {
+            const float c = ex2(sh_m[i] - Mu);  // 0 for an empty group
             const float4 o = sh_num[i][d4];
-            num.x += o.x;
-            num.y += o.y;
-            num.z += o.z;
-            num.w += o.w;
-            den += sh_den[i];
+            tot.x = fmaf(c, o.x, tot.x);
+            tot.y = fmaf(c, o.y, tot.y);
+            tot.z = fmaf(c, o.z, tot.z);
+            tot.w = fmaf(c, o.w, tot.w);
+            dt = fmaf(c, sh_den[i], dt);
         }
-        const float inv = den > 0.f ? 1.f / den : 0.f;
+        const float inv = dt > 0.f ? 1.f / dt : 0.f;
         reinterpret_cast<float4*>(outp)[d4] =
-            make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+            make_float4(tot.x * inv, tot.y * inv, tot.z * inv, tot.w * inv);
     }
 }
 
@@ -463,12 +521,13 @@ cudaError_t run(AttendParams p, int num_sms, cudaStream_t stream, int* launched)
     int blocks = num_sms * occ;
     if (blocks > kMaxAttendChunks) blocks = kMaxAttendChunks;
     p.num_chunks = blocks;  // chunk count (one chunk per CTA)
-    attend_kernel<D, NW, STAGES><<<blocks, NW * 32, smem, stream>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(attend_kernel<D, NW, STAGES>, dim3(blocks), dim3(NW * 32), smem,
+                               stream, p);
     if (e != cudaSuccess) return e;
-    merge_kernel<D><<<dim3(p.batch * p.hkv, p.group), kMergeGroups * D / 4, 0, stream>>>(p);
+    e = launch_pdl(merge_kernel<D>, dim3(p.batch * p.hkv, p.group), dim3(kMergeGroups * D / 4), 0,
+                   stream, p);
     if (launched) *launched += 2;
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace
@@ -476,7 +535,8 @@ cudaError_t run(AttendParams p, int num_sms, cudaStream_t stream, int* launched)
 cudaError_t launch_attend(AttendParams p, int head_dim, int num_sms, cudaStream_t stream,
                           int* launched) {
     if (p.batch * p.hkv == 0) return cudaSuccess;
-    if (head_dim == 128) return run<128, 4, 3>(p, num_sms, stream, launched);
+    // D=128: 4 warps x 2 stages x 8 KB = 64 KB per CTA, three CTAs per SM
+    if (head_dim == 128) return run<128, 4, 2>(p, num_sms, stream, launched);
     return run<256, 4, 3>(p, num_sms, stream, launched);
 }
 

@@ -4,9 +4,30 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "slc_device.cuh"
 
 namespace slc {
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the preceding kernel in the stream is still running; it calls
+// grid_dep_wait() before touching anything that kernel produces.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Upper bound on the number of attention CTAs (chunks) of one launch; sizes
 // the split-partial workspace (slot = unit + chunk index).
@@ -38,18 +59,27 @@ struct ScoreParams {
     const void* meta;
     const int32_t* block_table;
     const int32_t* seq_lens;
-    float* scores;  // [B][Hkv][max_pages]
+    float* scores;    // [B][Hkv][max_pages]
+    float* tile_max;  // nullable: [B][Hkv][tile_stride], max score per 16 candidates
     unsigned* status;
     int batch, hq, hkv, group, max_pages, num_pages, prefix, window;
+    int tile_stride;
 };
 
 struct SelectParams {
     const float* scores;
+    const float* tile_max;  // nullable (then computed from the scores)
     const int32_t* seq_lens;
     int32_t* selected;  // [B][Hkv][budget]
     unsigned* status;
     int batch, hkv, max_pages, prefix, window, budget;
+    int tile_stride;
 };
+
+// Candidates per selection tile and the row stride of the tile-maximum
+// array (a multiple of 4 floats).
+constexpr int kSelTile = 16;
+inline int tile_stride_of(int max_pages) { return ((max_pages + kSelTile - 1) / kSelTile + 3) / 4 * 4; }
 
 struct AttendParams {
     const void* q;
@@ -70,7 +100,7 @@ struct AttendParams {
 
 // Workspace carve-up shared by the API and the size query.
 struct WorkspaceLayout {
-    size_t scores, selected, part_acc, part_ml, total;
+    size_t scores, tile_max, selected, part_acc, part_ml, total;
 };
 WorkspaceLayout workspace_layout(int batch, int hq, int hkv, int head_dim, int max_pages,
                                  int budget);

@@ -43,6 +43,8 @@ __device__ __forceinline__ uint4 shfl_xor4(uint4 v, int m) {
 // piece of k, chunk c >= D/8 a piece of v.
 template <int D>
 __global__ void __launch_bounds__(128) kv_append_kernel(KvAppendParams p) {
+    grid_dep_wait();
+    grid_dep_launch();
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp >= p.batch * p.hkv) return;
@@ -144,10 +146,8 @@ cudaError_t launch_kv_append(const KvAppendParams& p, int head_dim, cudaStream_t
     const int threads = 128;
     const int blocks = (warps * 32 + threads - 1) / threads;
     if (head_dim == 128)
-        kv_append_kernel<128><<<blocks, threads, 0, stream>>>(p);
-    else
-        kv_append_kernel<256><<<blocks, threads, 0, stream>>>(p);
-    return cudaGetLastError();
+        return launch_pdl(kv_append_kernel<128>, dim3(blocks), dim3(threads), 0, stream, p);
+    return launch_pdl(kv_append_kernel<256>, dim3(blocks), dim3(threads), 0, stream, p);
 }
 
 cudaError_t launch_build_meta(const BuildMetaParams& p, int head_dim, int num_sms,
