@@ -55,6 +55,18 @@ def rank_info():
             int(os.environ.get("LOCAL_RANK", 0)))
 
 
+def max_over_ranks(x, device=None):
+    """The maximum of a float over all ranks (identity without a process
+    group).  Timing only: the decode path itself exchanges nothing."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def page_ranges(L, prefix, window):
     """Page ranges of the method (pages [0,np) prefix, [np,ws) candidates,
     [ws,n) window) -- used here only to count algorithmic bytes."""
@@ -305,11 +317,7 @@ def run_ours(args, rank, world, local):
     if world > 1:
         dist.barrier()
     step_ms = [s.elapsed_time(e) for s, e in ev]
-    total_ms = sum(step_ms)
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     assert slc.device_status() == 0
     ms_per_step = total_ms / K
     us_step = ms_per_step * 1e3
@@ -385,11 +393,7 @@ def run_ours(args, rank, world, local):
         outh.copy_(W64.out, non_blocking=True)
         e.record()
     torch.cuda.synchronize()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in e2e_ev)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in e2e_ev), dev)
     h2d = (qh[0].numel() * 2 + knh[0].numel() * 2 + vnh[0].numel() * 2 + posh[0].numel() * 4
            + lenh[0].numel() * 4)
     e2e = {"value": round(e2e_ms * 1e3 / K / world, 3), "unit": UNIT,
