@@ -170,6 +170,38 @@ SLC_API int slc_dense_decode(const void *q, const slc_cache_t *cache, const int3
                      int32_t num_q_heads, float scale, float *out, void *workspace,
                      size_t workspace_bytes, slc_stream_t stream);
 
+/* Bytes of device scratch that slc_sparse_decode_static owns (16 MiB). */
+#define SLC_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* slc_sparse_decode for callers that cannot allocate device memory: the
+ * same decode step (same arguments and results, minus the workspace), with
+ * its scratch taken from a fixed SLC_STATIC_SCRATCH_BYTES array that lives
+ * in the library's device code.  This entry point has no counterpart in the
+ * paper; it exists because some callers cannot allocate device memory at
+ * all -- for instance a plugin running inside a host framework that owns
+ * every byte of GPU memory through its own pool and forbids direct
+ * cudaMalloc -- so they cannot provide the workspace slc_sparse_decode
+ * needs.
+ *
+ * - Allocates nothing: no cudaMalloc/cudaFree and no allocating library
+ *   call.  Every GPU that loads the library holds the array until the
+ *   process exits.
+ * - Shapes whose workspace (slc_workspace_size) exceeds
+ *   SLC_STATIC_SCRATCH_BYTES are rejected with SLC_ERR_WORKSPACE before any
+ *   CUDA call.
+ * - The first call on a device looks up the array's device address (once
+ *   per device, with that device current); make that first call before
+ *   any stream capture.
+ * - Every call on a device shares the one array, and the array keeps the
+ *   last call's contents (nothing in it needs to start at zero).  Calls
+ *   whose executions overlap on the GPU -- on different streams, or from
+ *   different host threads -- race on it: serialise them. */
+SLC_API int slc_sparse_decode_static(const void *q, const slc_cache_t *cache,
+                             const int32_t *block_table, int32_t max_pages_per_seq,
+                             const int32_t *seq_lens, int32_t batch, int32_t num_q_heads,
+                             int32_t prefix, int32_t window, int32_t budget, float scale,
+                             float *out, int32_t *selected_out, slc_stream_t stream);
+
 /* Synchronise `stream`, read the current GPU's status word into *status
  * (host pointer; SLC_STATUS_* bits), then clear it.  Returns SLC_OK, or
  * SLC_ERR_CUDA. */

@@ -304,6 +304,55 @@ int slc_dense_decode(const void* q, const slc_cache_t* cache, const int32_t* blo
                   stream);
 }
 
+// ----------------------------------------------------------------------
+// Decode without any allocation: the workspace is a fixed device array.
+// Host code must not pass `slc_static_scratch` itself to a kernel (in host
+// code it names a host-side stand-in); its device address is looked up per
+// device below.
+static __device__ __align__(256) unsigned char slc_static_scratch[SLC_STATIC_SCRATCH_BYTES];
+
+static void* g_static_scratch[slc::kMaxDevices];
+static std::mutex g_static_mutex;
+
+// Device address of the scratch array on the current device (looked up
+// once per device, with that device current).
+static int static_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return note_cuda(e, "static scratch");
+    if (dev < 0 || dev >= slc::kMaxDevices) return SLC_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_static_mutex);
+    if (!g_static_scratch[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, slc_static_scratch);
+        if (e != cudaSuccess) return note_cuda(e, "static scratch");
+        g_static_scratch[dev] = ptr;
+    }
+    *out = g_static_scratch[dev];
+    return SLC_OK;
+}
+
+int slc_sparse_decode_static(const void* q, const slc_cache_t* cache, const int32_t* block_table,
+                             int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                             int32_t num_q_heads, int32_t prefix, int32_t window, int32_t budget,
+                             float scale, float* out, int32_t* selected_out,
+                             slc_stream_t stream) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if ((rc = check_heads(cache, num_q_heads))) return rc;
+    if (batch < 0 || max_pages_per_seq <= 0 || budget < 0) return SLC_ERR_INVALID_ARG;
+    const size_t need = workspace_layout(batch, num_q_heads, cache->num_kv_heads,
+                                         cache->head_dim, max_pages_per_seq, budget)
+                            .total;
+    if (need > SLC_STATIC_SCRATCH_BYTES) return SLC_ERR_WORKSPACE;
+    if (batch == 0) return SLC_OK;
+    void* scratch = nullptr;
+    if ((rc = static_scratch(&scratch))) return rc;
+    return slc_sparse_decode(q, cache, block_table, max_pages_per_seq, seq_lens, batch,
+                             num_q_heads, prefix, window, budget, scale, out, selected_out,
+                             scratch, SLC_STATIC_SCRATCH_BYTES, stream);
+}
+
 int slc_device_status(int32_t* status, slc_stream_t stream) {
     if (!status) return SLC_ERR_INVALID_ARG;
     DeviceInfo* dev;
