@@ -84,10 +84,10 @@ WorkspaceLayout workspace_layout(int batch, int hq, int hkv, int head_dim, int m
     WorkspaceLayout w{};
     const size_t units = (size_t)batch * hkv;
     const size_t group = (size_t)(hq / hkv);
-    const size_t slots = units + kMaxAttendChunks;
+    const size_t slots = fused_slots(units);
     size_t off = 0;
-    w.scores = off;
-    off = round_up(off + units * max_pages * sizeof(float), 256);
+    w.scores = off;  // by page (score_pages), or by candidate in rows of 16 * tile_stride
+    off = round_up(off + units * (size_t)tile_stride_of(max_pages) * 16 * sizeof(float), 256);
     w.tile_max = off;
     off = round_up(off + units * tile_stride_of(max_pages) * sizeof(float), 256);
     w.selected = off;
@@ -96,6 +96,8 @@ WorkspaceLayout workspace_layout(int batch, int hq, int hkv, int head_dim, int m
     off = round_up(off + slots * group * head_dim * sizeof(float), 256);
     w.part_ml = off;
     off = round_up(off + slots * group * sizeof(float2), 256);
+    w.counters = off;
+    off = round_up(off + (2 + 2 * units) * sizeof(int), 256);
     w.total = off;
     return w;
 }
@@ -234,21 +236,6 @@ static int decode(int mode, const void* q, const slc_cache_t* cache,
     if (scale <= 0.f) scale = 1.f / sqrtf((float)D);
     int32_t* sel = selected_out ? selected_out : reinterpret_cast<int32_t*>(ws + w.selected);
     cudaError_t e = cudaSuccess;
-    if (mode == 1 && budget > 0) {
-        float* scores = reinterpret_cast<float*>(ws + w.scores);
-        float* tmax = reinterpret_cast<float*>(ws + w.tile_max);
-        const int ts = tile_stride_of(max_pages_per_seq);
-        ScoreParams sp{q,           cache->meta, block_table, seq_lens,
-                       scores,      tmax,        dev->status, batch,
-                       num_q_heads, hkv,         num_q_heads / hkv, max_pages_per_seq,
-                       cache->num_pages, prefix, window, ts};
-        e = launch_score(sp, D, dev->num_sms, stream);
-        if (e != cudaSuccess) return note_cuda(e, "score_pages");
-        SelectParams lp{scores, tmax,   seq_lens, sel,    dev->status, batch, hkv,
-                        max_pages_per_seq, prefix, window, budget, ts};
-        e = launch_select(lp, stream);
-        if (e != cudaSuccess) return note_cuda(e, "select_pages");
-    }
     AttendParams ap{};
     ap.q = q;
     ap.k_cache = cache->k_cache;
@@ -266,11 +253,27 @@ static int decode(int mode, const void* q, const slc_cache_t* cache,
     ap.group = num_q_heads / hkv;
     ap.max_pages = max_pages_per_seq;
     ap.num_pages = cache->num_pages;
-    ap.sparse = sparse ? 1 : 0;
+    ap.list = sparse ? kListSparse : kListDense;
     ap.prefix = prefix;
     ap.window = window;
     ap.budget = sparse ? budget : 0;
     ap.scale_log2 = scale * 1.4426950408889634f;
+    if (mode == 1) {
+        float* scores = reinterpret_cast<float*>(ws + w.scores);
+        float* tmax = reinterpret_cast<float*>(ws + w.tile_max);
+        const int ts = tile_stride_of(max_pages_per_seq);
+        FusedParams fp{};
+        fp.sc = ScoreParams{q,           cache->meta, block_table, seq_lens,
+                            scores,      tmax,        dev->status, batch,
+                            num_q_heads, hkv,         num_q_heads / hkv, max_pages_per_seq,
+                            cache->num_pages, prefix, window, ts, 16 * ts};
+        fp.se = SelectParams{scores, tmax,   seq_lens, sel,    dev->status, batch, hkv,
+                             max_pages_per_seq, prefix, window, budget, ts, 16 * ts};
+        fp.at = ap;
+        fp.counters = reinterpret_cast<int*>(ws + w.counters);
+        e = launch_sparse_fused(fp, D, dev->num_sms, stream);
+        return e == cudaSuccess ? SLC_OK : note_cuda(e, "sparse decode");
+    }
     e = launch_attend(ap, D, dev->num_sms, stream, nullptr);
     return e == cudaSuccess ? SLC_OK : note_cuda(e, "attend/merge");
 }

@@ -32,272 +32,13 @@
 // (r, c) covers physical dims 8*(c+4m)..8*(c+4m)+7, identically for Q and K.
 // For P V, thread (r, c) owns dims (D/8)*r .. (D/8)*r + D/8 - 1, read as
 // 16-byte vectors and paired across tokens with byte permutes.
-#include "slc_internal.h"
+#include "slc_attend_impl.cuh"
 
 namespace slc {
 
 namespace {
 
-constexpr uint32_t kWaitLimit = 1u << 22;  // bounded mbarrier polls
-
-struct Ring {
-    uint8_t* tiles;  // STAGES x (K tile, V tile)
-    uint64_t* bars;  // STAGES
-    int* nvalid;     // STAGES
-};
-
-// A unit's list: dense = pages 0..n-1; sparse = prefix pages, window pages,
-// then the selected pages (forced pages first, so they need no selection).
-__device__ __forceinline__ bool list_is_selected(const AttendParams& p, const PageRanges& r,
-                                                 int i) {
-    return p.sparse && i >= r.np + (r.n - r.ws);
-}
-
-// Logical page of list position i of a unit (and whether it is sane).
-__device__ __forceinline__ int list_page(const AttendParams& p, int u, const PageRanges& r,
-                                         int i, bool* ok) {
-    *ok = true;
-    if (!p.sparse || i < r.np) return i;
-    const int nwin = r.n - r.ws;
-    if (i < r.np + nwin) return r.ws + (i - r.np);
-    const int j = p.selected[(long long)u * p.budget + (i - r.np - nwin)];
-    if (j < r.np || j >= r.ws) {
-        *ok = false;
-        return 0;
-    }
-    return j;
-}
-
-// Physical page and valid-token count of list position i of unit u;
-// (0, 0) for an entry that fails its range check (flagged, then skipped).
-__device__ __forceinline__ void resolve_page(const AttendParams& p, int u, int b,
-                                             const PageRanges& r, int L, int i, int* phys,
-                                             int* nv) {
-    bool ok;
-    const int j = list_page(p, u, r, i, &ok);
-    *phys = 0;
-    *nv = 0;
-    if (!ok) {
-        atomicOr(p.status, SLC_STATUS_BAD_SELECTION);
-        return;
-    }
-    const int ph = p.block_table[(long long)b * p.max_pages + j];
-    if (ph < 0 || ph >= p.num_pages) {
-        atomicOr(p.status, SLC_STATUS_BAD_PAGE);
-        return;
-    }
-    *phys = ph;
-    *nv = min(kPage, L - j * kPage);
-}
-
-// Lane 0: bulk-copy the K and V tiles of (phys, h) into ring stage `stage`.
-template <int D>
-__device__ __forceinline__ void issue_kv(const AttendParams& p, const Ring& ring, int stage,
-                                         int h, int phys, int nv) {
-    constexpr uint32_t TILE = kPage * D * 2;
-    ring.nvalid[stage] = nv;
-    uint64_t* bar = ring.bars + stage;
-    mbar_arrive_expect_tx(bar, 2 * TILE);
-    const long long off = ((long long)phys * p.hkv + h) * (kPage * D);
-    uint8_t* dst = ring.tiles + stage * 2 * TILE;
-    bulk_g2s(dst, static_cast<const __nv_bfloat16*>(p.k_cache) + off, TILE, bar);
-    bulk_g2s(dst + TILE, static_cast<const __nv_bfloat16*>(p.v_cache) + off, TILE, bar);
-}
-
-// Per-warp partial state: the running max of head r_ (log2 units), this
-// thread's share of the running sum, and the O^T accumulators of heads 2c,
-// 2c+1 over dims (D/8)*r_ .. (D/8)*r_ + D/8 - 1.
-template <int D>
-struct WarpState {
-    float m, l;
-    float acc[D / 16][4];
-};
-
-// Attend list positions i0, i0 + stride, ... < i1 of unit u with this warp's
-// ring.  `it` counts the warp's ring uses (stage = it % STAGES).  `ok` turns
-// false if a bounded wait gave up; the warp then drains its copies in flight
-// and skips all further work (it still reaches every CTA barrier).
-template <int D, int STAGES>
-__device__ void warp_attend(const AttendParams& p, const Ring& ring, uint32_t& it, bool& ok,
-                            int u, int i0, int i1, int stride, WarpState<D>& st) {
-    constexpr int TILE_W = kPage * D / 2;  // 32-bit words per tile
-    constexpr int ROW_W = D / 2;           // words per token row
-    constexpr int KS = D / 16;             // k-steps of Q K^T, m-blocks of V^T P^T
-    const int lane = threadIdx.x & 31;
-    const int r_ = lane >> 2, c_ = lane & 3;
-    const int b = u / p.hkv, h = u % p.hkv;
-    const int G = p.group;
-    st.m = -INFINITY;
-    st.l = 0.f;
-#pragma unroll
-    for (int i = 0; i < KS; ++i) st.acc[i][0] = st.acc[i][1] = st.acc[i][2] = st.acc[i][3] = 0.f;
-    const int npg = i1 > i0 ? (i1 - i0 + stride - 1) / stride : 0;
-    if (!ok || npg == 0) return;
-    const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
-    const PageRanges r = page_ranges(L, p.prefix, p.window);
-
-    // page ids of this warp's pages, 32 at a time: lane t holds page k0 + t.
-    // Selected pages come from the preceding (selection) kernel: wait for
-    // it only when a batch holds one.
-    int id_phys = 0, id_nv = 0;
-    auto load_ids = [&](int k0) {
-        const int k = k0 + lane;
-        const bool sel = k < npg && list_is_selected(p, r, i0 + k * stride);
-        if (__any_sync(0xffffffffu, sel)) grid_dep_wait();
-        if (k < npg) resolve_page(p, u, b, r, L, i0 + k * stride, &id_phys, &id_nv);
-    };
-    load_ids(0);
-    __syncwarp();  // this warp's earlier reads of the ring are done
-    fence_proxy_async_smem();
-    for (int k = 0; k < STAGES && k < npg; ++k) {
-        const int ph = __shfl_sync(0xffffffffu, id_phys, k);
-        const int nv = __shfl_sync(0xffffffffu, id_nv, k);
-        if (lane == 0) issue_kv<D>(p, ring, (it + k) % STAGES, h, ph, nv);
-    }
-    __syncwarp();
-
-    // query fragments (rows >= G and rows 8..15 are zero)
-    uint32_t qa[KS][2];
-    if (r_ < G) {
-        const uint4* qrow = reinterpret_cast<const uint4*>(
-            static_cast<const __nv_bfloat16*>(p.q) + ((long long)b * p.hq + h * G + r_) * D);
-#pragma unroll
-        for (int m = 0; m < D / 32; ++m) {
-            const uint4 v = __ldg(qrow + c_ + 4 * m);
-            qa[2 * m][0] = v.x;
-            qa[2 * m][1] = v.y;
-            qa[2 * m + 1][0] = v.z;
-            qa[2 * m + 1][1] = v.w;
-        }
-    } else {
-#pragma unroll
-        for (int k = 0; k < KS; ++k) qa[k][0] = qa[k][1] = 0u;
-    }
-
-    for (int k = 0; k < npg; ++k) {
-        const uint32_t use = it + k;
-        const int stage = use % STAGES;
-        if (!mbar_wait_bounded(ring.bars + stage, (use / STAGES) & 1u, kWaitLimit)) {
-            if (lane == 0) {
-                atomicOr(p.status, SLC_STATUS_WAIT_TIMEOUT);
-                for (int kk = k; kk < npg && kk < k + STAGES; ++kk) {
-                    const uint32_t u2 = it + kk;
-                    mbar_wait_bounded(ring.bars + u2 % STAGES, (u2 / STAGES) & 1u, kWaitLimit);
-                }
-            }
-            __syncwarp();
-            ok = false;
-            return;
-        }
-        const uint32_t* Kw = reinterpret_cast<const uint32_t*>(ring.tiles) + stage * 2 * TILE_W;
-        const uint32_t* Vw = Kw + TILE_W;
-        const int nv = ring.nvalid[stage];
-
-        // S = Q K^T for tokens nb*8 + (0..7)
-        float s[2][4];
-#pragma unroll
-        for (int nb = 0; nb < 2; ++nb) {
-            s[nb][0] = s[nb][1] = s[nb][2] = s[nb][3] = 0.f;
-            const uint32_t* krow = Kw + (nb * 8 + r_) * ROW_W;
-#pragma unroll
-            for (int m = 0; m < D / 32; ++m) {
-                const uint4 kv = lds128(krow + (c_ + 4 * m) * 4);
-                mma_bf16(s[nb], qa[2 * m][0], 0u, qa[2 * m][1], 0u, kv.x, kv.y);
-                mma_bf16(s[nb], qa[2 * m + 1][0], 0u, qa[2 * m + 1][1], 0u, kv.z, kv.w);
-            }
-        }
-        // this thread: head r_, tokens 2c, 2c+1, 8+2c, 9+2c
-        const int t0 = 2 * c_;
-        float x[4];
-        x[0] = t0 < nv ? s[0][0] * p.scale_log2 : -INFINITY;
-        x[1] = t0 + 1 < nv ? s[0][1] * p.scale_log2 : -INFINITY;
-        x[2] = t0 + 8 < nv ? s[1][0] * p.scale_log2 : -INFINITY;
-        x[3] = t0 + 9 < nv ? s[1][1] * p.scale_log2 : -INFINITY;
-        float pmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-        pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 1));
-        pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 2));
-        const float m_new = fmaxf(st.m, pmax);
-        const float m_use = m_new == -INFINITY ? 0.f : m_new;
-        const float alpha = ex2(st.m - m_use);
-        float pr[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) pr[e] = ex2(x[e] - m_use);
-        st.l = st.l * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
-        st.m = m_new;
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {  // some head's maximum moved
-            const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * c_);
-            const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * c_ + 4);
-#pragma unroll
-            for (int i = 0; i < KS; ++i) {
-                st.acc[i][0] *= a0;
-                st.acc[i][1] *= a1;
-                st.acc[i][2] *= a0;
-                st.acc[i][3] *= a1;
-            }
-        }
-        // P^T fragments (tokens 2c,2c+1 / 2c+8,2c+9 of head r_), hi + lo
-        const uint32_t bh0 = pack_bf16x2(pr[0], pr[1]);
-        const uint32_t bh1 = pack_bf16x2(pr[2], pr[3]);
-        const uint32_t bl0 = pack_bf16x2(pr[0] - bf16_lo(bh0), pr[1] - bf16_hi(bh0));
-        const uint32_t bl1 = pack_bf16x2(pr[2] - bf16_lo(bh1), pr[3] - bf16_hi(bh1));
-
-        // V rows of tokens 2c, 2c+1, 2c+8, 2c+9, dims (D/8)*r_ .. +D/8
-        constexpr int WPT = D / 16;  // words per token per thread
-        uint32_t vw[4][WPT];
-#pragma unroll
-        for (int tt = 0; tt < 4; ++tt) {
-            const int tok = t0 + (tt & 1) + (tt >> 1) * 8;
-            const uint32_t* vrow = Vw + tok * ROW_W + WPT * r_;
-#pragma unroll
-            for (int q4 = 0; q4 < WPT / 4; ++q4) {
-                const uint4 v = lds128(vrow + 4 * q4);
-                vw[tt][4 * q4 + 0] = v.x;
-                vw[tt][4 * q4 + 1] = v.y;
-                vw[tt][4 * q4 + 2] = v.z;
-                vw[tt][4 * q4 + 3] = v.w;
-            }
-        }
-        if (nv < kPage) {  // partial page: zero slots past the length (may hold NaN)
-#pragma unroll
-            for (int tt = 0; tt < 4; ++tt) {
-                const bool live = t0 + (tt & 1) + (tt >> 1) * 8 < nv;
-#pragma unroll
-                for (int i = 0; i < WPT; ++i) vw[tt][i] = live ? vw[tt][i] : 0u;
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < KS; ++i) {
-            const uint32_t a0r = __byte_perm(vw[0][i], vw[1][i], 0x5410);
-            const uint32_t a1r = __byte_perm(vw[0][i], vw[1][i], 0x7632);
-            const uint32_t a2r = __byte_perm(vw[2][i], vw[3][i], 0x5410);
-            const uint32_t a3r = __byte_perm(vw[2][i], vw[3][i], 0x7632);
-            mma_bf16(st.acc[i], a0r, a1r, a2r, a3r, bh0, bh1);
-            mma_bf16(st.acc[i], a0r, a1r, a2r, a3r, bl0, bl1);
-        }
-        __syncwarp();
-        const int kn = k + STAGES;
-        if (kn < npg) {  // refill this stage (warp-uniform branch)
-            if ((kn & 31) == 0) load_ids(kn);
-            const int ph = __shfl_sync(0xffffffffu, id_phys, kn & 31);
-            const int nv = __shfl_sync(0xffffffffu, id_nv, kn & 31);
-            if (lane == 0) {
-                fence_proxy_async_smem();
-                issue_kv<D>(p, ring, stage, h, ph, nv);
-            }
-        }
-    }
-    it += npg;
-    // full sum of head r_ (the four threads of a quad hold parts of it)
-    st.l += __shfl_xor_sync(0xffffffffu, st.l, 1);
-    st.l += __shfl_xor_sync(0xffffffffu, st.l, 2);
-}
-
-__device__ __forceinline__ int list_len(const AttendParams& p, int b) {
-    const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
-    const PageRanges r = page_ranges(L, p.prefix, p.window);
-    if (!p.sparse) return r.n;
-    return r.np + min(p.budget, r.ws - r.np) + (r.n - r.ws);
-}
+using namespace attn;
 
 // One CTA per chunk of the concatenated page lists.  For every unit piece
 // of the chunk, the CTA's warps take its pages round-robin, then combine
@@ -307,12 +48,8 @@ template <int D, int NW, int STAGES>
 __global__ void __launch_bounds__(NW * 32) attend_kernel(AttendParams p) {
     constexpr int TILE = kPage * D * 2;
     constexpr int RING = STAGES * 2 * TILE;
-    constexpr int KS = D / 16;
-    constexpr int DPT = D / 8;
-    static_assert(RING >= (kMaxGroup * D + 2 * kMaxGroup) * 4, "ring holds a warp partial");
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r_ = lane >> 2, c_ = lane & 3;
     Ring ring;
     ring.tiles = smem + warp * RING;
     ring.bars = reinterpret_cast<uint64_t*>(smem + NW * RING) + warp * STAGES;
@@ -327,78 +64,11 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttendParams p) {
     auto len_of = [&](int b) { return list_len(p, b); };
     const long long total = total_units(p.batch, p.hkv, len_of);
     const long long cpp = (total + gridDim.x - 1) / gridDim.x;
-    long long s = (long long)blockIdx.x * cpp;
+    const long long s = (long long)blockIdx.x * cpp;
     const long long e = min(total, s + cpp);
-    if (s >= e) return;  // uniform across the CTA
-    int u;
-    long long ustart;
-    locate_unit(s, p.batch, p.hkv, len_of, &u, &ustart);
     uint32_t it = 0;
     bool ok = true;
-    const int G = p.group;
-    WarpState<D> st;
-    while (s < e) {
-        const int len = list_len(p, u / p.hkv);
-        if (len == 0) {
-            ++u;
-            continue;
-        }
-        const int i0 = (int)(s - ustart);
-        const int i1 = (int)(min(e, ustart + len) - ustart);
-        warp_attend<D, STAGES>(p, ring, it, ok, u, i0 + warp, i1, NW, st);
-
-        // combine the NW warp partials through shared memory; global writes
-        // only after the preceding kernel has completed
-        grid_dep_wait();
-        __syncthreads();  // every warp is done with its ring
-        float* wacc = reinterpret_cast<float*>(smem + warp * RING);  // [G][D]
-        float2* wml = reinterpret_cast<float2*>(wacc + kMaxGroup * D);  // [G]
-        if (c_ == 0 && r_ < G) wml[r_] = make_float2(st.m, st.l);
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int head = 2 * c_ + hh;
-            if (head < G) {
-                float4* dst = reinterpret_cast<float4*>(wacc + head * D + DPT * r_);
-#pragma unroll
-                for (int i2 = 0; i2 < KS / 2; ++i2)
-                    dst[i2] = make_float4(st.acc[2 * i2][hh], st.acc[2 * i2][2 + hh],
-                                          st.acc[2 * i2 + 1][hh], st.acc[2 * i2 + 1][2 + hh]);
-            }
-        }
-        __syncthreads();
-        const long long slot = (long long)u + blockIdx.x;
-        for (int item = threadIdx.x; item < G * (D / 4); item += NW * 32) {
-            const int g = item / (D / 4), d4 = item % (D / 4);
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < NW; ++w) {
-                const float2 ml = reinterpret_cast<const float2*>(
-                    reinterpret_cast<const float*>(smem + w * RING) + kMaxGroup * D)[g];
-                M = fmaxf(M, ml.x);
-            }
-            const float Mu = M == -INFINITY ? 0.f : M;
-            float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-            float den = 0.f;
-#pragma unroll
-            for (int w = 0; w < NW; ++w) {
-                const float* wa = reinterpret_cast<const float*>(smem + w * RING);
-                const float2 ml = reinterpret_cast<const float2*>(wa + kMaxGroup * D)[g];
-                const float wt = ex2(ml.x - Mu);
-                const float4 a = reinterpret_cast<const float4*>(wa + g * D)[d4];
-                num.x = fmaf(wt, a.x, num.x);
-                num.y = fmaf(wt, a.y, num.y);
-                num.z = fmaf(wt, a.z, num.z);
-                num.w = fmaf(wt, a.w, num.w);
-                den = fmaf(wt, ml.y, den);
-            }
-            reinterpret_cast<float4*>(p.part_acc + (slot * G + g) * D)[d4] = num;
-            if (d4 == 0) p.part_ml[slot * G + g] = make_float2(M, den);
-        }
-        __syncthreads();  // the rings are reused by the next piece
-        s = ustart + len;
-        ustart = s;
-        ++u;
-    }
+    attend_range<D, NW, STAGES>(p, smem, ring, it, ok, s, e, blockIdx.x, 0, [](int) {});
 }
 
 // Merge of the CTA partials of one (unit, query head): slots unit + chunk

@@ -59,11 +59,12 @@ struct ScoreParams {
     const void* meta;
     const int32_t* block_table;
     const int32_t* seq_lens;
-    float* scores;    // [B][Hkv][max_pages]
+    float* scores;    // [B][Hkv][max_pages] by page, or by candidate (cand_stride)
     float* tile_max;  // nullable: [B][Hkv][tile_stride], max score per 16 candidates
     unsigned* status;
     int batch, hq, hkv, group, max_pages, num_pages, prefix, window;
     int tile_stride;
+    int cand_stride;  // 0: scores indexed by page; else rows of cand_stride by candidate
 };
 
 struct SelectParams {
@@ -74,12 +75,16 @@ struct SelectParams {
     unsigned* status;
     int batch, hkv, max_pages, prefix, window, budget;
     int tile_stride;
+    int cand_stride;  // as ScoreParams::cand_stride
 };
 
 // Candidates per selection tile and the row stride of the tile-maximum
 // array (a multiple of 4 floats).
 constexpr int kSelTile = 16;
 inline int tile_stride_of(int max_pages) { return ((max_pages + kSelTile - 1) / kSelTile + 3) / 4 * 4; }
+
+// Page list attended per unit (see slc_attend_impl.cuh).
+enum : int { kListDense = 0, kListSparse = 1, kListForced = 2, kListSelected = 3 };
 
 struct AttendParams {
     const void* q;
@@ -93,15 +98,28 @@ struct AttendParams {
     float* out;               // [B][Hq][D]
     unsigned* status;
     int batch, hq, hkv, group, max_pages, num_pages;
-    int sparse, prefix, window, budget;
+    int list;  // kListDense, kListSparse, kListForced or kListSelected
+    int prefix, window, budget;
     float scale_log2;  // softmax scale * log2(e)
     int num_chunks;    // chunks of the attention launch (one per CTA)
 };
 
 // Workspace carve-up shared by the API and the size query.
 struct WorkspaceLayout {
-    size_t scores, tile_max, selected, part_acc, part_ml, total;
+    size_t scores, tile_max, selected, part_acc, part_ml, counters, total;
 };
+
+// Fused sparse decode: scoring, selection and attention in one persistent
+// grid, then the merge (slc_fused.cu).
+struct FusedParams {
+    ScoreParams sc;
+    SelectParams se;
+    AttendParams at;  // list is set per kernel
+    int* counters;    // 2 + 2U ints (U units), zeroed by the launcher
+};
+// Split-partial slots of the fused decode: two phases of at most
+// units + kMaxAttendChunks slots each.
+inline size_t fused_slots(size_t units) { return 2 * (units + kMaxAttendChunks); }
 WorkspaceLayout workspace_layout(int batch, int hq, int hkv, int head_dim, int max_pages,
                                  int budget);
 
@@ -110,6 +128,10 @@ cudaError_t launch_build_meta(const BuildMetaParams& p, int head_dim, int num_sm
                               cudaStream_t stream);
 cudaError_t launch_score(const ScoreParams& p, int head_dim, int num_sms, cudaStream_t stream);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
+// Score, select and attend in one fused kernel, then merge (counters
+// zeroed first); sparse_decode's path.
+cudaError_t launch_sparse_fused(const FusedParams& p, int head_dim, int num_sms,
+                                cudaStream_t stream);
 // Attention over the list of each unit (dense: all pages; sparse: prefix,
 // selected, window), then the merge of the per-warp partials into out.
 cudaError_t launch_attend(AttendParams p, int head_dim, int num_sms, cudaStream_t stream,
