@@ -31,8 +31,9 @@ __all__ = [
 
 PAGE = 16
 
-# kernels one call launches (sparse: two fused kernels; dense and attend: attend, merge)
-KERNELS_PER_CALL = {"sparse_decode": 2, "dense_decode": 2, "sparse_attend": 2, "kv_append": 1,
+# kernels one call launches (sparse: score with forced attention, select, attend,
+# merge; dense and attend: attend, merge)
+KERNELS_PER_CALL = {"sparse_decode": 4, "dense_decode": 2, "sparse_attend": 2, "kv_append": 1,
                     "build_page_meta": 1, "score_pages": 1, "select_pages": 1}
 
 STATUS_BITS = {1: "bad page", 2: "bad length", 4: "bad selection", 8: "wait timeout"}

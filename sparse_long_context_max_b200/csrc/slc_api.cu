@@ -86,18 +86,14 @@ WorkspaceLayout workspace_layout(int batch, int hq, int hkv, int head_dim, int m
     const size_t group = (size_t)(hq / hkv);
     const size_t slots = fused_slots(units);
     size_t off = 0;
-    w.scores = off;  // by page (score_pages), or by candidate in rows of 16 * tile_stride
-    off = round_up(off + units * (size_t)tile_stride_of(max_pages) * 16 * sizeof(float), 256);
-    w.tile_max = off;
-    off = round_up(off + units * tile_stride_of(max_pages) * sizeof(float), 256);
+    w.scores = off;  // by candidate, in rows of cand_stride_of(max_pages)
+    off = round_up(off + units * (size_t)cand_stride_of(max_pages) * sizeof(float), 256);
     w.selected = off;
     off = round_up(off + units * (size_t)(budget > 0 ? budget : 1) * sizeof(int32_t), 256);
     w.part_acc = off;
     off = round_up(off + slots * group * head_dim * sizeof(float), 256);
     w.part_ml = off;
     off = round_up(off + slots * group * sizeof(float2), 256);
-    w.counters = off;
-    off = round_up(off + (2 + 2 * units) * sizeof(int), 256);
     w.total = off;
     return w;
 }
@@ -181,7 +177,7 @@ int slc_score_pages(const void* q, const slc_cache_t* cache, const int32_t* bloc
     DeviceInfo* dev;
     if ((rc = device_info(&dev))) return rc;
     ScoreParams p{q,           cache->meta, block_table, seq_lens,
-                  scores,      nullptr,     dev->status, batch,
+                  scores,      dev->status, batch,
                   num_q_heads, cache->num_kv_heads, num_q_heads / cache->num_kv_heads,
                   max_pages_per_seq, cache->num_pages, prefix, window, 0};
     cudaError_t e = launch_score(p, cache->head_dim, dev->num_sms, stream);
@@ -200,7 +196,7 @@ int slc_select_pages(const float* scores, int32_t num_kv_heads, int32_t max_page
     DeviceInfo* dev;
     int rc;
     if ((rc = device_info(&dev))) return rc;
-    SelectParams p{scores, nullptr, seq_lens, selected, dev->status, batch, num_kv_heads,
+    SelectParams p{scores, seq_lens, selected, dev->status, batch, num_kv_heads,
                    max_pages_per_seq, prefix, window, budget, 0};
     cudaError_t e = launch_select(p, stream);
     return e == cudaSuccess ? SLC_OK : note_cuda(e);
@@ -260,17 +256,15 @@ static int decode(int mode, const void* q, const slc_cache_t* cache,
     ap.scale_log2 = scale * 1.4426950408889634f;
     if (mode == 1) {
         float* scores = reinterpret_cast<float*>(ws + w.scores);
-        float* tmax = reinterpret_cast<float*>(ws + w.tile_max);
-        const int ts = tile_stride_of(max_pages_per_seq);
+        const int cs = cand_stride_of(max_pages_per_seq);
         FusedParams fp{};
         fp.sc = ScoreParams{q,           cache->meta, block_table, seq_lens,
-                            scores,      tmax,        dev->status, batch,
+                            scores,      dev->status, batch,
                             num_q_heads, hkv,         num_q_heads / hkv, max_pages_per_seq,
-                            cache->num_pages, prefix, window, ts, 16 * ts};
-        fp.se = SelectParams{scores, tmax,   seq_lens, sel,    dev->status, batch, hkv,
-                             max_pages_per_seq, prefix, window, budget, ts, 16 * ts};
+                            cache->num_pages, prefix, window, cs};
+        fp.se = SelectParams{scores, seq_lens, sel,    dev->status, batch, hkv,
+                             max_pages_per_seq, prefix, window, budget, cs};
         fp.at = ap;
-        fp.counters = reinterpret_cast<int*>(ws + w.counters);
         e = launch_sparse_fused(fp, D, dev->num_sms, stream);
         return e == cudaSuccess ? SLC_OK : note_cuda(e, "sparse decode");
     }

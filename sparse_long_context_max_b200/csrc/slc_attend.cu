@@ -68,7 +68,8 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttendParams p) {
     const long long e = min(total, s + cpp);
     uint32_t it = 0;
     bool ok = true;
-    attend_range<D, NW, STAGES>(p, smem, ring, it, ok, s, e, blockIdx.x, 0, [](int) {});
+    attend_range<D, NW, STAGES>(p, smem, ring, it, ok, s, e, blockIdx.x, p.slot_base,
+                                [](int) {});
 }
 
 // Merge of the CTA partials of one (unit, query head): slots unit + chunk
@@ -176,7 +177,7 @@ constexpr int attend_smem() {
 }
 
 template <int D, int NW, int STAGES>
-cudaError_t run(AttendParams p, int num_sms, cudaStream_t stream, int* launched) {
+cudaError_t run(AttendParams& p, int num_sms, cudaStream_t stream, bool merge, int* launched) {
     constexpr int smem = attend_smem<D, NW, STAGES>();
     static int occ = 0;
     if (occ == 0) {
@@ -193,7 +194,7 @@ cudaError_t run(AttendParams p, int num_sms, cudaStream_t stream, int* launched)
     p.num_chunks = blocks;  // chunk count (one chunk per CTA)
     cudaError_t e = launch_pdl(attend_kernel<D, NW, STAGES>, dim3(blocks), dim3(NW * 32), smem,
                                stream, p);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess || !merge) return e;
     e = launch_pdl(merge_kernel<D>, dim3(p.batch * p.hkv, p.group), dim3(kMergeGroups * D / 4), 0,
                    stream, p);
     if (launched) *launched += 2;
@@ -205,9 +206,17 @@ cudaError_t run(AttendParams p, int num_sms, cudaStream_t stream, int* launched)
 cudaError_t launch_attend(AttendParams p, int head_dim, int num_sms, cudaStream_t stream,
                           int* launched) {
     if (p.batch * p.hkv == 0) return cudaSuccess;
+    p.slot_base = 0;
     // D=128: 4 warps x 2 stages x 8 KB = 64 KB per CTA, three CTAs per SM
-    if (head_dim == 128) return run<128, 4, 2>(p, num_sms, stream, launched);
-    return run<256, 4, 3>(p, num_sms, stream, launched);
+    if (head_dim == 128) return run<128, 4, 2>(p, num_sms, stream, true, launched);
+    return run<256, 4, 3>(p, num_sms, stream, true, launched);
+}
+
+cudaError_t launch_attend_partials(AttendParams& p, int head_dim, int num_sms,
+                                   cudaStream_t stream) {
+    if (p.batch * p.hkv == 0) return cudaSuccess;
+    if (head_dim == 128) return run<128, 4, 2>(p, num_sms, stream, false, nullptr);
+    return run<256, 4, 3>(p, num_sms, stream, false, nullptr);
 }
 
 }  // namespace slc

@@ -190,27 +190,6 @@ __device__ __forceinline__ void grid_dep_launch() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// Acquire load / release store of a flag or counter in global memory
-// (GPU scope).
-__device__ __forceinline__ int ld_acquire(const int* p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release(int* p, int v) {
-    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Bounded wait until *p >= target: gives up after `limit` polls (about
-// 100 ns apart) and returns false.
-__device__ __forceinline__ bool wait_at_least(const int* p, int target, uint32_t limit) {
-    for (uint32_t i = 0; i < limit; ++i) {
-        if (ld_acquire(p) >= target) return true;
-        __nanosleep(64);
-    }
-    return false;
-}
-
 __device__ __forceinline__ uint4 lds128(const void* p) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"

@@ -1,36 +1,26 @@
-// Fused sparse decode step of one layer: page scoring, per-unit top-k
-// selection, split-KV attention over prefix + window + selected pages
-// ("Hybrid LLM Decoding 2.2x Faster at 256k, No Retraining", section "The
-// method: sliding window + prefix + query-aware pages, searched per
-// layer") in one persistent kernel, then the log-sum-exp merge.
+// Sparse decode step of one layer ("Hybrid LLM Decoding 2.2x Faster at
+// 256k, No Retraining", section "The method: sliding window + prefix +
+// query-aware pages, searched per layer"): four kernels chained by
+// programmatic dependent launch, none of whose CTAs ever waits for another.
 //
-// The CTAs of decode_kernel take two roles.
-//   Selectors (the first S CTAs): selector s owns units s, s+S, ...; for
-//     each it waits until every tile of the unit is scored, selects the
-//     unit's pages and raises the unit's selection flag.
-//   Streamers (the others) take work from two ticket counters:
-//     1. per warp, scoring tiles (16 candidate pages of one unit), numbered
-//        unit after unit so that units finish scoring one after another;
-//        a warp counts each scored tile for its unit;
-//     2. per CTA, attention chunks: first over the forced lists (prefix
-//        pages, then window pages) of all units, then over the selected
-//        pages of all units, unit after unit.  Before a unit's selected
-//        pages the CTA waits for the unit's selection flag.
-// Selection is latency-bound and runs beside the streams; by the time
-// the streamers reach a unit's selected pages its selection is normally
-// done.  Every wait is bounded: on timeout the kernel sets the
-// wait-timeout status bit and goes on, so a fault shows as a status error,
-// never as a hang.  Waits cannot deadlock: a streamer waits only after all
-// scoring tiles have been claimed by running warps that never wait, and the
-// selectors are the lowest-numbered CTAs, resident first.
+//   1. score_forced_kernel (persistent): every CTA first attends one chunk
+//      of the forced lists (prefix pages, then window pages) of all units,
+//      cut into about one chunk per CTA; then every warp scores candidate
+//      tiles (16 pages of one unit) strided over the grid's warps.  Both
+//      halves stream HBM; the forced attention needs no selection, so it
+//      rides along with the scoring, and the scores are written last, so
+//      the selection finds them in L2.
+//   2. select_kernel (slc_select.cu): one CTA per unit, from the scores the
+//      first kernel left.
+//   3. attend_kernel (slc_attend.cu) over the selected pages of all units.
+//   4. merge_kernel: log-sum-exp merge of both kernels' partials per (unit,
+//      query head).
 //
 // Partials: forced chunk c of unit u goes to slot u + c, selected chunk c
-// to slot U + chunks_forced + u + c (U units); a chunk covers consecutive
-// list positions, so each slot is written once.  merge_kernel then combines
-// the slots of every (unit, query head), one CTA each.
+// to slot U + kMaxAttendChunks + u + c (U units); a chunk covers
+// consecutive list positions, so each slot is written once.
 #include "slc_attend_impl.cuh"
 #include "slc_score_impl.cuh"
-#include "slc_select_impl.cuh"
 
 namespace slc {
 
@@ -61,24 +51,7 @@ struct FusedGeom : FusedCfg<D> {
     static constexpr int DATA_SCORE = B::NW * SRING;
     static constexpr int DATA = DATA_ATT > DATA_SCORE ? DATA_ATT : DATA_SCORE;
     static constexpr int SMEM = DATA + B::NW * B::STAGES * (8 + 4);
-    static_assert(DATA >= sel::kLiveBytes + 1024 * 8, "selection needs room for survivors");
 };
-
-constexpr int kChunkPages = 16;          // target pages per attention chunk
-constexpr uint32_t kFlagWait = 1u << 22;  // bounded polls of a flag (~0.4 s)
-
-// Counters (zeroed before the kernel): [0] scoring ticket, [1] attention
-// ticket, [2, 2+U) tiles scored per unit, [2+U, 2+2U) selection flags.
-struct Counters {
-    int* score_ticket;
-    int* attn_ticket;
-    int* tiles_done;
-    int* sel_done;
-};
-__device__ __forceinline__ Counters counters_of(const FusedParams& p) {
-    const int U = p.sc.batch * p.sc.hkv;
-    return Counters{p.counters, p.counters + 1, p.counters + 2, p.counters + 2 + U};
-}
 
 // Tiles to score for sequence b: none when the budget keeps every
 // candidate (the selection is then the candidate range itself).
@@ -89,16 +62,17 @@ __device__ __forceinline__ int unit_tiles(const ScoreParams& p, int budget, int 
     return ncand > budget ? (ncand + scr::kTilePages - 1) / scr::kTilePages : 0;
 }
 
-// Chunking of one list kind: total positions, chunk count, positions per
-// chunk.  Warp-wide; every kernel computes it identically.
+// Chunking of the forced lists into about `target` chunks: total positions,
+// chunk count, positions per chunk.  Warp-wide; the scoring and merge
+// kernels compute it identically.
 struct Chunking {
     long long total, chunks, cpp;
 };
-__device__ __forceinline__ Chunking chunking(const AttendParams& at) {
+__device__ __forceinline__ Chunking forced_chunking(const AttendParams& at, int target) {
     auto len_of = [&](int b) { return attn::list_len(at, b); };
     Chunking c;
     c.total = total_units(at.batch, at.hkv, len_of);
-    long long n = (c.total + kChunkPages - 1) / kChunkPages;
+    long long n = c.total < target ? c.total : target;
     if (n > kMaxAttendChunks) n = kMaxAttendChunks;
     c.cpp = n > 0 ? (c.total + n - 1) / n : 1;
     c.chunks = n > 0 ? (c.total + c.cpp - 1) / c.cpp : 0;
@@ -118,52 +92,21 @@ struct TileRef {
     bool valid;
 };
 
+// Scoring by one warp: tiles w, w + nw, w + 2 nw, ... (w this warp's index
+// among the grid's nw warps).  Tiles are numbered sequence after sequence
+// and, within a sequence, (tile, kv head): at any moment the warps sweep
+// consecutive tiles, and the kv heads' metadata rows of a page (adjacent
+// in memory) are read together.
 template <int D>
-__device__ void selector(const FusedParams& p, const Counters& ctr, uint8_t* smem,
-                         sel::Scratch<FusedGeom<D>::NTHR>& sc, int first, int stride) {
-    using F = FusedGeom<D>;
-    const ScoreParams& ps = p.sc;
-    const int budget = p.se.budget;
-    const int U = ps.batch * ps.hkv;
-    for (int u = first; u < U; u += stride) {
-        const int b = u / ps.hkv;
-        const int nt = unit_tiles(ps, budget, b);
-        if (nt == 0) {  // every candidate is kept
-            const int L = checked_len(ps.seq_lens, b, ps.max_pages, ps.status);
-            const PageRanges r = page_ranges(L, ps.prefix, ps.window);
-            const int ncand = r.ws - r.np;
-            int32_t* out = p.se.selected + (long long)u * budget;
-            for (int i = threadIdx.x; i < budget; i += F::NTHR) out[i] = i < ncand ? r.np + i : -1;
-        } else {
-            if (threadIdx.x == 0 && !wait_at_least(ctr.tiles_done + u, nt, kFlagWait))
-                atomicOr(ps.status, SLC_STATUS_WAIT_TIMEOUT);
-            __syncthreads();
-            sel::select_unit<F::NTHR>(p.se, u, smem, F::DATA, sc);
-        }
-        __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0) st_release(ctr.sel_done + u, 1);
-    }
-}
-
-// Scoring phase of one streamer warp: claim tiles until none is left.
-template <int D>
-__device__ void score_tiles(const FusedParams& p, const Counters& ctr, uint8_t* sring,
-                            int n_tiles) {
+__device__ void score_tiles(const FusedParams& p, uint8_t* sring, int n_tiles, int w, int nw) {
     using F = FusedGeom<D>;
     using TG = scr::TileGeom<D>;
     constexpr int NT = F::NT;
     const ScoreParams& ps = p.sc;
     const int budget = p.se.budget;
-    const int lane = threadIdx.x & 31;
-    // tickets: lane 0 claims one ahead; the value is read a tile later
-    auto claim = [&]() { return lane == 0 ? atomicAdd(ctr.score_ticket, 1) : 0; };
-    auto bcast = [&](int v) { return __shfl_sync(0xffffffffu, v, 0); };
-    int cur = bcast(claim());
-    if (cur >= n_tiles) return;
-    int nxt = bcast(claim());
-    // forward-only cursor over units (a warp's tickets grow)
-    int cu = 0, cstart = 0, ccount = unit_tiles(ps, budget, 0);
+    if (w >= n_tiles) return;
+    // forward-only cursor over sequences (a warp's tiles grow)
+    int cb = 0, cstart = 0, ccount = unit_tiles(ps, budget, 0) * ps.hkv;
     PageRanges cr = page_ranges(checked_len(ps.seq_lens, 0, ps.max_pages, ps.status),
                                 ps.prefix, ps.window);
     auto locate = [&](int g) {
@@ -172,14 +115,14 @@ __device__ void score_tiles(const FusedParams& p, const Counters& ctr, uint8_t* 
         if (!t.valid) return t;
         while (g >= cstart + ccount) {
             cstart += ccount;
-            ++cu;
-            const int b = cu / ps.hkv;
-            cr = page_ranges(checked_len(ps.seq_lens, b, ps.max_pages, ps.status), ps.prefix,
+            ++cb;
+            cr = page_ranges(checked_len(ps.seq_lens, cb, ps.max_pages, ps.status), ps.prefix,
                              ps.window);
-            ccount = unit_tiles(ps, budget, b);
+            ccount = unit_tiles(ps, budget, cb) * ps.hkv;
         }
-        t.u = cu;
-        t.jt = g - cstart;
+        const int k = g - cstart;
+        t.u = cb * ps.hkv + k % ps.hkv;
+        t.jt = k / ps.hkv;
         t.r = cr;
         return t;
     };
@@ -189,21 +132,12 @@ __device__ void score_tiles(const FusedParams& p, const Counters& ctr, uint8_t* 
         scr::copy_tile<D>(ps, t.u % ps.hkv, phys, sring + (issued % NT) * TG::TILE_B);
         ++issued;
     };
-    // A tile is counted for its unit one tile later, after a fence that
-    // then finds its score stores long completed (a fence right after them
-    // would stall the warp on their acknowledgement).
-    auto publish = [&](int u) {
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) atomicAdd(ctr.tiles_done + u, 1);
-    };
-    int wu = -1, done_u = -1;
-    float w[TG::CPL][8];
-    TileRef tcur = locate(cur);
+    int wu = -1;
+    float wt[TG::CPL][8];
+    TileRef tcur = locate(w);
     issue(tcur);
-    while (tcur.valid) {
-        const TileRef tnxt = locate(nxt);
-        const int after = tnxt.valid ? claim() : 0;
+    for (int g = w; tcur.valid; g += nw) {
+        const TileRef tnxt = locate(g + nw);
         bool nxt_issued = false;
         if (NT > 1 && tnxt.valid) {
             issue(tnxt);
@@ -213,30 +147,25 @@ __device__ void score_tiles(const FusedParams& p, const Counters& ctr, uint8_t* 
             cp_async_wait<1>();
         else
             cp_async_wait<0>();
-        if (done_u >= 0) publish(done_u);
         if (tcur.u != wu) {
             wu = tcur.u;
-            scr::load_weights<D>(ps, wu, w);
+            scr::load_weights<D>(ps, wu, wt);
         }
-        scr::score_tile<D>(ps, tcur.u, tcur.r, tcur.jt, sring + (consumed % NT) * TG::TILE_B, w);
+        scr::score_tile<D>(ps, tcur.u, tcur.r, tcur.jt, sring + (consumed % NT) * TG::TILE_B,
+                           wt);
         ++consumed;
-        done_u = tcur.u;
         tcur = tnxt;
-        nxt = tnxt.valid ? bcast(after) : n_tiles;
         if (tcur.valid && !nxt_issued) issue(tcur);
     }
-    publish(done_u);
     cp_async_wait<0>();
 }
 
 template <int D>
 __global__ void __launch_bounds__(FusedGeom<D>::NTHR, FusedGeom<D>::MINB)
-    decode_kernel(FusedParams p, int selectors) {
+    score_forced_kernel(FusedParams p) {
     using F = FusedGeom<D>;
     constexpr int NW = F::NW;
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ sel::Scratch<F::NTHR> sc;
-    __shared__ int sh_ticket;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     attn::Ring ring;
     ring.tiles = smem + warp * F::RING;
@@ -248,65 +177,37 @@ __global__ void __launch_bounds__(FusedGeom<D>::NTHR, FusedGeom<D>::MINB)
     }
     __syncwarp();
 
-    // q, metadata and the zeroed counters come from preceding work
+    // q and the metadata come from preceding work; partial slots may still
+    // be read by a preceding merge
     grid_dep_wait();
     grid_dep_launch();
 
-    const Counters ctr = counters_of(p);
-    if ((int)blockIdx.x < selectors) {
-        selector<D>(p, ctr, smem, sc, blockIdx.x, selectors);
-        return;
+    const AttendParams atF = with_list(p.at, kListForced);
+    const Chunking cf = forced_chunking(atF, p.forced_chunks);
+    uint32_t it = 0;
+    bool ok = true;
+    for (long long c = blockIdx.x; c < cf.chunks; c += gridDim.x) {
+        const long long s = c * cf.cpp;
+        attn::attend_range<D, NW, F::STAGES>(atF, smem, ring, it, ok, s, min(cf.total, s + cf.cpp),
+                                             c, 0, [](int) {});
     }
+    __syncthreads();  // the attention rings are idle: the data region turns to scoring rings
 
     const ScoreParams& ps = p.sc;
     const int budget = p.se.budget;
     auto tiles_of = [&](int b) { return unit_tiles(ps, budget, b); };
     const int n_tiles = budget > 0 ? (int)total_units(ps.batch, ps.hkv, tiles_of) : 0;
-    if (n_tiles > 0) score_tiles<D>(p, ctr, smem + warp * F::SRING, n_tiles);
-    __syncthreads();  // the scoring rings are idle: the data region turns to attention rings
-
-    const AttendParams atF = with_list(p.at, kListForced);
-    const AttendParams atS = with_list(p.at, kListSelected);
-    const Chunking cf = chunking(atF), cs = chunking(atS);
-    const long long n_tickets = cf.chunks + cs.chunks;
-    const long long base_s = (long long)ps.batch * ps.hkv + cf.chunks;
-    uint32_t it = 0;
-    bool ok = true;
-    auto wait_selection = [&](int u) {
-        if (threadIdx.x == 0 && !wait_at_least(ctr.sel_done + u, 1, kFlagWait))
-            atomicOr(ps.status, SLC_STATUS_WAIT_TIMEOUT);
-        __syncthreads();
-    };
-    if (threadIdx.x == 0) sh_ticket = atomicAdd(ctr.attn_ticket, 1);
-    __syncthreads();
-    long long t = sh_ticket;
-    while (t < n_tickets) {
-        // the next ticket is claimed now and published after the chunk
-        const int next = threadIdx.x == 0 ? atomicAdd(ctr.attn_ticket, 1) : 0;
-        if (t < cf.chunks) {
-            const long long s = t * cf.cpp;
-            attn::attend_range<D, NW, F::STAGES>(atF, smem, ring, it, ok, s,
-                                                 min(cf.total, s + cf.cpp), t, 0, [](int) {});
-        } else {
-            const long long c = t - cf.chunks;
-            const long long s = c * cs.cpp;
-            attn::attend_range<D, NW, F::STAGES>(atS, smem, ring, it, ok, s,
-                                                 min(cs.total, s + cs.cpp), c, base_s,
-                                                 wait_selection);
-        }
-        if (threadIdx.x == 0) sh_ticket = next;
-        __syncthreads();
-        t = sh_ticket;
-        __syncthreads();  // every thread has read sh_ticket
-    }
+    if (n_tiles > 0)
+        score_tiles<D>(p, smem + warp * F::SRING, n_tiles, blockIdx.x * NW + warp, gridDim.x * NW);
 }
 
 // Log-sum-exp merge of the split partials of one (unit, query head):
-//   out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k,  M = max_k m_k.
-// The block's threads split into kMergeGroups slot groups x D/4 dimension
+//   out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k,  M = max_k m_k,
+// over the forced-list slots and the selected-list slots of the unit.  The
+// block's threads split into kMergeGroups slot groups x D/4 dimension
 // quads; each group folds its slots with online rescaling, then the groups
 // combine in shared memory.
-constexpr int kMergeGroups = 4;
+constexpr int kMergeGroups = 8;
 
 template <int D>
 __global__ void __launch_bounds__(kMergeGroups * D / 4) merge_kernel(FusedParams p) {
@@ -323,22 +224,24 @@ __global__ void __launch_bounds__(kMergeGroups * D / 4) merge_kernel(FusedParams
     __shared__ float4 sh_num[kMergeGroups][V4];
     __shared__ float sh_den[kMergeGroups];
     if (tid < 32) {
-        const Chunking cf = chunking(atF), cs = chunking(atS);
+        const Chunking cf = forced_chunking(atF, p.forced_chunks);
+        auto len_sel = [&](int bb) { return attn::list_len(atS, bb); };
+        const long long totalS = total_units(atS.batch, atS.hkv, len_sel);
+        const long long cppS = totalS > 0 ? (totalS + p.at.num_chunks - 1) / p.at.num_chunks : 1;
         const long long sA = attn::unit_list_start(atF, u);
         const long long sB = attn::unit_list_start(atS, u);
         const int lenA = attn::list_len(atF, b), lenB = attn::list_len(atS, b);
-        const long long base_s = (long long)atF.batch * atF.hkv + cf.chunks;
         if (tid == 0) {
             sh_r[0] = lenA > 0 ? u + sA / cf.cpp : 0;
             sh_r[1] = lenA > 0 ? u + (sA + lenA - 1) / cf.cpp : -1;
-            sh_r[2] = lenB > 0 ? base_s + u + sB / cs.cpp : 0;
-            sh_r[3] = lenB > 0 ? base_s + u + (sB + lenB - 1) / cs.cpp : -1;
+            sh_r[2] = lenB > 0 ? p.at.slot_base + u + sB / cppS : 0;
+            sh_r[3] = lenB > 0 ? p.at.slot_base + u + (sB + lenB - 1) / cppS : -1;
         }
     }
     __syncthreads();
     const long long a0 = sh_r[0], a1 = sh_r[1], b0 = sh_r[2], b1 = sh_r[3];
     const long long na = a1 - a0 + 1, nb = b1 - b0 + 1;
-    grid_dep_wait();  // the partials come from the decode kernel
+    grid_dep_wait();  // the partials come from the attention kernels
     float M = -INFINITY, den = 0.f;
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
@@ -394,29 +297,35 @@ __global__ void __launch_bounds__(kMergeGroups * D / 4) merge_kernel(FusedParams
 }
 
 template <int D>
-cudaError_t run_fused(const FusedParams& p, int num_sms, cudaStream_t stream) {
+cudaError_t run_sparse(const FusedParams& p, int num_sms, cudaStream_t stream) {
     using F = FusedGeom<D>;
     static int occ = 0;
     if (occ == 0) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D>,
+        cudaError_t e = cudaFuncSetAttribute(score_forced_kernel<D>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM);
         if (e == cudaSuccess)
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<D>, F::NTHR,
-                                                              F::SMEM);
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, score_forced_kernel<D>,
+                                                              F::NTHR, F::SMEM);
         if (e != cudaSuccess) return e;
         if (occ < 1) occ = 1;
     }
     const int U = p.sc.batch * p.sc.hkv;
     const int grid = num_sms * occ;
-    // selectors: one per unit up to 16, never more than a quarter of the grid
-    int selectors = p.se.budget > 0 ? (U < 16 ? U : 16) : 0;
-    if (selectors > grid / 4) selectors = grid / 4;
-    cudaError_t e = cudaMemsetAsync(p.counters, 0, (size_t)(2 + 2 * U) * sizeof(int), stream);
+    FusedParams q = p;
+    q.forced_chunks = grid;  // about one chunk per CTA
+    cudaError_t e = launch_pdl(score_forced_kernel<D>, dim3(grid), dim3(F::NTHR), F::SMEM, stream,
+                               q);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(decode_kernel<D>, dim3(grid), dim3(F::NTHR), F::SMEM, stream, p, selectors);
-    if (e != cudaSuccess) return e;
+    q.at.list = kListSelected;
+    q.at.slot_base = (long long)U + kMaxAttendChunks;
+    q.at.num_chunks = 1;
+    if (p.se.budget > 0) {
+        e = launch_select(p.se, stream);
+        if (e == cudaSuccess) e = launch_attend_partials(q.at, D, num_sms, stream);
+        if (e != cudaSuccess) return e;
+    }
     return launch_pdl(merge_kernel<D>, dim3(U, p.at.group), dim3(kMergeGroups * D / 4), 0, stream,
-                      p);
+                      q);
 }
 
 }  // namespace
@@ -424,8 +333,8 @@ cudaError_t run_fused(const FusedParams& p, int num_sms, cudaStream_t stream) {
 cudaError_t launch_sparse_fused(const FusedParams& p, int head_dim, int num_sms,
                                 cudaStream_t stream) {
     if (p.sc.batch * p.sc.hkv == 0) return cudaSuccess;
-    if (head_dim == 128) return run_fused<128>(p, num_sms, stream);
-    return run_fused<256>(p, num_sms, stream);
+    if (head_dim == 128) return run_sparse<128>(p, num_sms, stream);
+    return run_sparse<256>(p, num_sms, stream);
 }
 
 }  // namespace slc

@@ -59,29 +59,25 @@ struct ScoreParams {
     const void* meta;
     const int32_t* block_table;
     const int32_t* seq_lens;
-    float* scores;    // [B][Hkv][max_pages] by page, or by candidate (cand_stride)
-    float* tile_max;  // nullable: [B][Hkv][tile_stride], max score per 16 candidates
+    float* scores;  // [B][Hkv][max_pages] by page, or by candidate (cand_stride)
     unsigned* status;
     int batch, hq, hkv, group, max_pages, num_pages, prefix, window;
-    int tile_stride;
     int cand_stride;  // 0: scores indexed by page; else rows of cand_stride by candidate
 };
 
 struct SelectParams {
-    const float* scores;
-    const float* tile_max;  // nullable (then computed from the scores)
+    const float* scores;  // as ScoreParams::scores (cand_stride)
     const int32_t* seq_lens;
     int32_t* selected;  // [B][Hkv][budget]
     unsigned* status;
     int batch, hkv, max_pages, prefix, window, budget;
-    int tile_stride;
-    int cand_stride;  // as ScoreParams::cand_stride
+    int cand_stride;
 };
 
-// Candidates per selection tile and the row stride of the tile-maximum
-// array (a multiple of 4 floats).
+// Candidates per scoring tile, and the row stride of candidate-indexed
+// scores (a multiple of 64 floats: 16-byte aligned rows and tiles).
 constexpr int kSelTile = 16;
-inline int tile_stride_of(int max_pages) { return ((max_pages + kSelTile - 1) / kSelTile + 3) / 4 * 4; }
+inline int cand_stride_of(int max_pages) { return (max_pages + 63) / 64 * 64; }
 
 // Page list attended per unit (see slc_attend_impl.cuh).
 enum : int { kListDense = 0, kListSparse = 1, kListForced = 2, kListSelected = 3 };
@@ -102,23 +98,24 @@ struct AttendParams {
     int prefix, window, budget;
     float scale_log2;  // softmax scale * log2(e)
     int num_chunks;    // chunks of the attention launch (one per CTA)
+    long long slot_base;  // this launch's partials: slot slot_base + unit + chunk
 };
 
 // Workspace carve-up shared by the API and the size query.
 struct WorkspaceLayout {
-    size_t scores, tile_max, selected, part_acc, part_ml, counters, total;
+    size_t scores, selected, part_acc, part_ml, total;
 };
 
-// Fused sparse decode: scoring, selection and attention in one persistent
-// grid, then the merge (slc_fused.cu).
+// Sparse decode step (slc_fused.cu): scoring with the prefix/window
+// attention in one grid, selection, selected-page attention, merge.
 struct FusedParams {
     ScoreParams sc;
     SelectParams se;
     AttendParams at;  // list is set per kernel
-    int* counters;    // 2 + 2U ints (U units), zeroed by the launcher
+    int forced_chunks;  // target chunk count of the prefix/window attention
 };
-// Split-partial slots of the fused decode: two phases of at most
-// units + kMaxAttendChunks slots each.
+// Split-partial slots of the sparse decode: two attention launches of at
+// most units + kMaxAttendChunks slots each.
 inline size_t fused_slots(size_t units) { return 2 * (units + kMaxAttendChunks); }
 WorkspaceLayout workspace_layout(int batch, int hq, int hkv, int head_dim, int max_pages,
                                  int budget);
@@ -128,13 +125,17 @@ cudaError_t launch_build_meta(const BuildMetaParams& p, int head_dim, int num_sm
                               cudaStream_t stream);
 cudaError_t launch_score(const ScoreParams& p, int head_dim, int num_sms, cudaStream_t stream);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
-// Score, select and attend in one fused kernel, then merge (counters
-// zeroed first); sparse_decode's path.
+// sparse_decode's path: four kernels chained by programmatic dependent
+// launch (score + forced attention, select, selected attention, merge).
 cudaError_t launch_sparse_fused(const FusedParams& p, int head_dim, int num_sms,
                                 cudaStream_t stream);
 // Attention over the list of each unit (dense: all pages; sparse: prefix,
 // selected, window), then the merge of the per-warp partials into out.
 cudaError_t launch_attend(AttendParams p, int head_dim, int num_sms, cudaStream_t stream,
                           int* kernels_launched);
+// The attention alone: partials in slots p.slot_base + unit + chunk; sets
+// p.num_chunks (at most kMaxAttendChunks).
+cudaError_t launch_attend_partials(AttendParams& p, int head_dim, int num_sms,
+                                   cudaStream_t stream);
 
 }  // namespace slc

@@ -125,7 +125,7 @@ __device__ __forceinline__ void copy_tile(const ScoreParams& p, int h, int phys,
 }
 
 // Score the landed tile jt of unit u (rows in `tile`) and write the page
-// scores and, if p.tile_max is set, the tile maximum.
+// scores.
 template <int D>
 __device__ __forceinline__ void score_tile(const ScoreParams& p, int u, const PageRanges& r,
                                            int jt, const uint8_t* tile,
@@ -157,23 +157,14 @@ __device__ __forceinline__ void score_tile(const ScoreParams& p, int u, const Pa
     }
     acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
     const int j = r.np + jt * kTilePages + (lane >> 1);
-    float sc = -INFINITY;
-    if (j < r.ws) {
+    if (j < r.ws && (lane & 1) == 0) {
         // a page whose block-table entry failed its check scores -inf
         const int phys = p.block_table[(long long)(u / p.hkv) * p.max_pages + j];
-        sc = (phys < 0 || phys >= p.num_pages) ? -INFINITY : acc[0];
-        if ((lane & 1) == 0) {
-            if (p.cand_stride)
-                p.scores[(long long)u * p.cand_stride + (j - r.np)] = sc;
-            else
-                p.scores[(long long)u * p.max_pages + j] = sc;
-        }
-    }
-    if (p.tile_max) {
-#pragma unroll
-        for (int dist = 16; dist >= 2; dist >>= 1)
-            sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, dist));
-        if (lane == 0) p.tile_max[(long long)u * p.tile_stride + jt] = sc;
+        const float sc = (phys < 0 || phys >= p.num_pages) ? -INFINITY : acc[0];
+        if (p.cand_stride)
+            p.scores[(long long)u * p.cand_stride + (j - r.np)] = sc;
+        else
+            p.scores[(long long)u * p.max_pages + j] = sc;
     }
 }
 

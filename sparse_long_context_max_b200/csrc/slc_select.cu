@@ -1,38 +1,57 @@
-// Fixed-budget page selection kernel: one 256-thread CTA per (sequence, kv
-// head) unit runs the exact two-level selection of slc_select_impl.cuh
-// ("Accelerating Long-Context Decoding in Large-Scale Hybrid LLMs Without
-// Retraining", abstract: a fixed budget of the most relevant tokens).
+// Fixed-budget page selection kernel: one 1024-thread CTA per (sequence, kv
+// head) unit runs the register-resident exact selection of
+// slc_select_impl.cuh ("Accelerating Long-Context Decoding in Large-Scale
+// Hybrid LLMs Without Retraining", abstract: a fixed budget of the most
+// relevant tokens).
 #include "slc_select_impl.cuh"
 
 namespace slc {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 1024;
 constexpr int kSurvivorCap = 8192;  // survivors held in shared memory
-constexpr int kSelectSmem = sel::kLiveBytes + kSurvivorCap * 8;
 
-__global__ void __launch_bounds__(kThreads) select_kernel(SelectParams p) {
+// Dynamic shared memory: the unit's scores (KPT per thread), then the
+// survivors (key and index each).
+template <int KPT>
+constexpr int select_smem() {
+    return kThreads * KPT * 4 + kSurvivorCap * 8;
+}
+
+template <int KPT>
+__global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectParams p) {
     __shared__ sel::Scratch<kThreads> sc;
-    extern __shared__ __align__(16) uint8_t buf[];
+    __shared__ uint64_t bar;
+    extern __shared__ __align__(128) uint32_t smem[];
+    float* stage = reinterpret_cast<float*>(smem);
+    uint32_t* surv = smem + kThreads * KPT;
     grid_dep_wait();  // the scores come from the preceding kernel
     grid_dep_launch();
-    sel::select_unit<kThreads>(p, blockIdx.x, buf, kSelectSmem, sc);
+    sel::select_unit<kThreads, KPT>(p, blockIdx.x, sc, surv, kSurvivorCap, stage, &bar);
+}
+
+template <int KPT>
+cudaError_t launch(const SelectParams& p, cudaStream_t stream) {
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(select_kernel<KPT>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             select_smem<KPT>());
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    return launch_pdl(select_kernel<KPT>, dim3(p.batch * p.hkv), dim3(kThreads),
+                      select_smem<KPT>(), stream, p);
 }
 
 }  // namespace
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
     if (p.batch * p.hkv == 0) return cudaSuccess;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(
-            select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelectSmem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
-    return launch_pdl(select_kernel, dim3(p.batch * p.hkv), dim3(kThreads), kSelectSmem, stream,
-                      p);
+    // candidates per unit are at most max_pages (<= kMaxCandidates)
+    if (p.max_pages <= 16 * kThreads) return launch<16>(p, stream);
+    return launch<32>(p, stream);
 }
 
 }  // namespace slc

@@ -1,49 +1,36 @@
-// Fixed-budget page selection of one (sequence, kv head) unit by one CTA,
-// shared by the selection kernel (slc_select.cu) and the fused sparse
-// decode (slc_fused.cu).  Keeps the budget candidate pages with the highest
-// scores, equal scores going to the lower page index, and emits them in
-// ascending page order ("Accelerating Long-Context Decoding in Large-Scale
-// Hybrid LLMs Without Retraining", abstract: a fixed budget of the most
-// relevant tokens).
+// Fixed-budget page selection of one (sequence, kv head) unit by one CTA
+// ("Accelerating Long-Context Decoding in Large-Scale Hybrid LLMs Without
+// Retraining", abstract: a fixed budget of the most relevant tokens): keep
+// the budget (k) candidate pages with the highest scores, equal scores going
+// to the lower page index, and emit them in ascending page order.
 //
-// Scores become order-preserving uint32 keys.  Exact selection in two
-// levels, built for latency (few dependent memory round trips, few block
-// barriers):
-//   1. the maximum key of every 16-candidate tile (written by the scoring
-//      code, or computed here from the scores): one round trip;
-//   2. tau <= the k-th largest tile maximum (k = budget; 0 when there are
-//      fewer tiles than the budget).  The k tiles whose maxima are >= that
-//      value hold k distinct pages >= tau, so tau <= T, the k-th largest
-//      page key: every selected page is >= tau.  The radix search for tau
-//      stops after two digits, at the smallest key with the digits found,
-//      which is still such a bound;
-//   3. the live tiles (maximum >= tau) are listed in index order and their
-//      scores read, two tiles per thread per round trip; the pages >= tau
-//      (typically little more than the budget) are compacted in index order
-//      into shared memory;
-//   4. an exact radix select over those survivors finds T and how many keys
+// Built for latency.  The CTA holds every candidate score of the unit in
+// registers (thread t: candidates t*KPT .. t*KPT+KPT-1, brought in by one
+// bulk copy) as order-preserving uint32 keys, then:
+//   1. tau <= the k-th largest of the threads' maxima (0 when fewer than k
+//      threads hold candidates): the k threads with the largest maxima hold
+//      k distinct keys >= that value, so tau <= T, the k-th largest key,
+//      and every selected key is >= tau.  The radix search for tau works on
+//      one key per thread and may stop after two digits, at the smallest key
+//      with those digits, which is still such a bound;
+//   2. the keys >= tau (typically little more than k) are compacted, in
+//      index order, into shared memory;
+//   3. an exact radix select over those survivors finds T and how many keys
 //      equal to T to keep (the lowest-indexed ones), and an index-ordered
-//      scan writes the result.
-// If ties leave more survivors than shared memory holds, steps 3-4 stream
-// over every candidate instead, re-reading the scores (cached in L2).
+//      block scan writes the pages.
+// If ties leave more survivors than shared memory holds, step 3 runs on
+// the register-resident keys of every candidate instead.
 //
 // The radix select works on 8-bit digits from the highest bit where the
-// set's smallest and largest keys differ, so equal leading bits cost no
-// pass, and stops as soon as the chosen digit's bin holds exactly the keys
-// still wanted.  Scores and tile maxima are read through L2
-// (ld.global.cg): in the fused decode they are written by other CTAs of the
-// same grid.
+// set's smallest and largest keys differ (equal leading bits cost no pass)
+// and stops as soon as the chosen digit's bin holds exactly the keys still
+// wanted.
 #pragma once
 
 #include "slc_internal.h"
 
 namespace slc {
 namespace sel {
-
-constexpr int kTile = kSelTile;  // candidates per tile
-constexpr int kMaxTiles = kMaxCandidates / kTile;
-constexpr int kLiveBytes = kMaxTiles * (int)sizeof(int);  // live-tile list
-constexpr int kLivePerThread = 2;  // live tiles read per thread per round
 
 __device__ __forceinline__ uint32_t order_key(float f) {
     if (f == 0.f) f = 0.f;  // -0 and +0 tie
@@ -64,6 +51,7 @@ struct Scratch {
 template <int NTHR>
 __device__ __forceinline__ int block_excl_scan(int v, Scratch<NTHR>& sc, int* total) {
     constexpr int W = NTHR / 32;
+    static_assert(W <= 32, "one warp scans the warp totals");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int incl = warp_incl_scan(v);
     if (lane == 31) sc.scan[warp] = incl;
@@ -91,16 +79,17 @@ struct Kth {
 };
 
 // Radix search for the `want`-th largest key held by the block (1 <= want
-// <= count): thread t holds keys key_at(0 .. n_t-1) (n_t <= KMAX when
-// UNROLL: key_at reads a register array).  Key 0 never occurs.
-template <int NTHR, int KMAX, bool UNROLL, class KeyAt>
+// <= count): thread t holds keys key_at(0 .. n_t-1), n_t <= KMAX (KMAX > 0:
+// unrolled, key_at reads registers; KMAX == 0: a loop).  Key 0 never
+// occurs.
+template <int NTHR, int KMAX, class KeyAt>
 __device__ Kth radix_kth(int n_t, KeyAt key_at, int want, Scratch<NTHR>& sc, int max_passes) {
     constexpr int W = NTHR / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint32_t kmin = 0xffffffffu, kmax = 0u;
-    if (UNROLL) {
+    if (KMAX > 0) {
 #pragma unroll
-        for (int k = 0; k < KMAX; ++k)
+        for (int k = 0; k < (KMAX > 0 ? KMAX : 1); ++k)
             if (k < n_t) {
                 kmin = min(kmin, key_at(k));
                 kmax = max(kmax, key_at(k));
@@ -118,6 +107,7 @@ __device__ Kth radix_kth(int n_t, KeyAt key_at, int want, Scratch<NTHR>& sc, int
         sc.red_min[warp] = kmin;
         sc.red_max[warp] = kmax;
     }
+    for (int i = tid; i < 256; i += NTHR) sc.hist[0][i] = 0;
     __syncthreads();
     kmin = lane < W ? sc.red_min[lane] : 0xffffffffu;
     kmax = lane < W ? sc.red_max[lane] : 0u;
@@ -128,13 +118,12 @@ __device__ Kth radix_kth(int n_t, KeyAt key_at, int want, Scratch<NTHR>& sc, int
         __syncthreads();  // red_min/red_max are rewritten by the next call
         return r;
     }
+    const int n_warp = __reduce_max_sync(0xffffffffu, n_t);  // uniform trip count
     int hb = 31 - __clz(kmin ^ kmax);
     uint32_t mask = hb == 31 ? 0u : ~((2u << hb) - 1u);
     uint32_t prefix = kmin & mask;
     int remaining = want;
     int buf = 0;
-    for (int i = tid; i < 256; i += NTHR) sc.hist[0][i] = 0;
-    __syncthreads();
     for (int pass = 1;; ++pass) {
         const int shift = max(hb - 7, 0);
         const uint32_t dmask = (1u << (hb - shift + 1)) - 1u;
@@ -148,15 +137,12 @@ __device__ Kth radix_kth(int n_t, KeyAt key_at, int want, Scratch<NTHR>& sc, int
             const unsigned peers = __match_any_sync(0xffffffffu, bin);
             if (hit && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
         };
-        if (UNROLL) {
+        if (KMAX > 0) {
 #pragma unroll
-            for (int k = 0; k < KMAX; ++k) add(k < n_t, key_at(k));
+            for (int k = 0; k < (KMAX > 0 ? KMAX : 1); ++k)
+                if (k < n_warp) add(k < n_t, k < n_t ? key_at(k) : 0u);
         } else {
-            const int n_warp = __reduce_max_sync(0xffffffffu, n_t);  // uniform trip count
-            for (int k = 0; k < n_warp; ++k) {
-                const bool in = k < n_t;
-                add(in, in ? key_at(k) : 0u);
-            }
+            for (int k = 0; k < n_warp; ++k) add(k < n_t, k < n_t ? key_at(k) : 0u);
         }
         __syncthreads();
         if (warp == 0) {
@@ -214,45 +200,54 @@ __device__ Kth radix_kth(int n_t, KeyAt key_at, int want, Scratch<NTHR>& sc, int
     return r;
 }
 
-// Write, in index order, every key > T and the first `ties` keys == T.
-// Thread t's keys are consecutive in index order and precede thread t+1's.
-template <int NTHR, class KeyAt, class PageAt>
-__device__ void write_selected(int n_t, KeyAt key_at, PageAt page_at, uint32_t T, int ties,
-                               Scratch<NTHR>& sc, int32_t* out) {
+// Output positions, in index order, of every key > T and the first `ties`
+// keys == T: emit(position, k) for thread t's keys k (consecutive in index
+// order, preceding thread t+1's).
+template <int NTHR, int KMAX, class KeyAt, class Emit>
+__device__ void write_selected(int n_t, KeyAt key_at, uint32_t T, int ties, Scratch<NTHR>& sc,
+                               Emit emit) {
     int ngt = 0, neq = 0;
-    for (int k = 0; k < n_t; ++k) {
+    auto count = [&](int k) {
         const uint32_t v = key_at(k);
         ngt += v > T;
         neq += v == T;
+    };
+    if (KMAX > 0) {
+#pragma unroll
+        for (int k = 0; k < (KMAX > 0 ? KMAX : 1); ++k)
+            if (k < n_t) count(k);
+    } else {
+        for (int k = 0; k < n_t; ++k) count(k);
     }
     int total;
     const int excl = block_excl_scan<NTHR>((ngt << 16) | neq, sc, &total);
     int gt_before = excl >> 16, eq_before = excl & 0xffff;
-    for (int k = 0; k < n_t; ++k) {
+    auto place = [&](int k) {
         const uint32_t v = key_at(k);
         if (v > T) {
-            out[gt_before + min(eq_before, ties)] = page_at(k);
+            emit(gt_before + min(eq_before, ties), k);
             ++gt_before;
         } else if (v == T) {
-            if (eq_before < ties) out[gt_before + eq_before] = page_at(k);
+            if (eq_before < ties) emit(gt_before + eq_before, k);
             ++eq_before;
         }
+    };
+    if (KMAX > 0) {
+#pragma unroll
+        for (int k = 0; k < (KMAX > 0 ? KMAX : 1); ++k)
+            if (k < n_t) place(k);
+    } else {
+        for (int k = 0; k < n_t; ++k) place(k);
     }
 }
 
-// Select the pages of unit u (all threads of the CTA call it).  buf is
-// shared memory of buf_bytes (16-byte aligned): the live-tile list, then
-// the survivors.
-template <int NTHR>
-__device__ void select_unit(const SelectParams& p, int u, uint8_t* buf, int buf_bytes,
-                            Scratch<NTHR>& sc) {
-    constexpr int TPT = kMaxTiles / NTHR;  // tiles per thread
-    static_assert(TPT * NTHR == kMaxTiles && TPT % 4 == 0, "tile coverage");
-    int* live_tile = reinterpret_cast<int*>(buf);
-    const int surv_cap = (buf_bytes - kLiveBytes) / 8;
-    uint32_t* surv_key = reinterpret_cast<uint32_t*>(buf + kLiveBytes);
-    int32_t* surv_page = reinterpret_cast<int32_t*>(surv_key + surv_cap);
-
+// Select the pages of unit u (all NTHR threads of the CTA call it; the
+// unit's candidates must number at most NTHR * KPT).  surv is shared memory
+// for surv_cap survivors (keys, then candidate indices).
+template <int NTHR, int KPT>
+__device__ void select_unit(const SelectParams& p, int u, Scratch<NTHR>& sc, uint32_t* surv,
+                            int surv_cap, float* stage, uint64_t* bar) {
+    static_assert(KPT % 4 == 0, "16-byte loads");
     const int b = u / p.hkv;
     const int tid = threadIdx.x;
     const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
@@ -268,115 +263,83 @@ __device__ void select_unit(const SelectParams& p, int u, uint8_t* buf, int buf_
     for (int i = nsel + tid; i < p.budget; i += NTHR) out[i] = -1;
     if (nsel <= 0) return;
 
-    // candidate c's score: rows by candidate, or by page
-    const float* s = p.cand_stride ? p.scores + (long long)u * p.cand_stride
-                                   : p.scores + (long long)u * p.max_pages + r.np;
-    auto cand_key = [&](int c) { return order_key(__ldcg(s + c)); };
-    const int ntiles = (ncand + kTile - 1) / kTile;
-    const int t0 = tid * TPT;  // this thread's first tile
-    const int nt_own = max(0, min(TPT, ntiles - t0));
-
-    // 1. tile maxima
-    uint32_t tk[TPT];
-    if (p.tile_max) {
-        const float4* tm =
-            reinterpret_cast<const float4*>(p.tile_max + (long long)u * p.tile_stride);
+    // candidate c's score: rows by candidate (16-byte aligned), or by page
+    const int c0 = tid * KPT;
+    const int n_t = max(0, min(KPT, ncand - c0));
+    float f[KPT];
+    if (p.cand_stride) {
+        // one bulk copy (TMA engine) of the unit's row into `stage`: a single
+        // CTA cannot keep that many plain loads in flight
+        if (tid == 0) {
+            mbar_init(bar, 1);
+            fence_mbar_init();
+            const uint32_t bytes = (uint32_t)((ncand + 3) / 4) * 16;  // rows are padded
+            mbar_arrive_expect_tx(bar, bytes);
+            bulk_g2s(stage, p.scores + (long long)u * p.cand_stride, bytes, bar);
+        }
+        __syncthreads();  // the barrier is initialised
+        if (!mbar_wait_bounded(bar, 0, 1u << 22)) {
+            if (tid == 0) atomicOr(p.status, SLC_STATUS_WAIT_TIMEOUT);
+        }
+        const float4* s4 = reinterpret_cast<const float4*>(stage + c0);
 #pragma unroll
-        for (int q = 0; q < TPT / 4; ++q) {
-            const float4 a =
-                t0 + 4 * q < ntiles ? __ldcg(tm + t0 / 4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float v[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) tk[4 * q + k] = 4 * q + k < nt_own ? order_key(v[k]) : 0u;
+        for (int q = 0; q < KPT / 4; ++q) {
+            const float4 a = 4 * q < n_t ? s4[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+            f[4 * q] = a.x;
+            f[4 * q + 1] = a.y;
+            f[4 * q + 2] = a.z;
+            f[4 * q + 3] = a.w;
         }
     } else {
+        const float* s = p.scores + (long long)u * p.max_pages + r.np + c0;
 #pragma unroll
-        for (int k = 0; k < TPT; ++k) tk[k] = 0u;
-        for (int k = 0; k < nt_own; ++k) {
-            const int c0 = (t0 + k) * kTile;
-            uint32_t m = 0u;
-            uint32_t v[kTile];  // one tile's loads in flight together
+        for (int k = 0; k < KPT; ++k) f[k] = k < n_t ? __ldcg(s + k) : 0.f;
+    }
+    uint32_t key[KPT];
+    uint32_t kmax = 0u;
 #pragma unroll
-            for (int i = 0; i < kTile; ++i) v[i] = c0 + i < ncand ? cand_key(c0 + i) : 0u;
-#pragma unroll
-            for (int i = 0; i < kTile; ++i) m = max(m, v[i]);
-            // registers indexed by a runtime k: select into place
-#pragma unroll
-            for (int kk = 0; kk < TPT; ++kk)
-                if (kk == k) tk[kk] = m;
-        }
+    for (int k = 0; k < KPT; ++k) {
+        key[k] = k < n_t ? order_key(f[k]) : 0u;
+        kmax = max(kmax, key[k]);
     }
 
-    // 2. tau: at most the nsel-th largest tile maximum (0 keeps every page)
+    // 1. tau from the threads' maxima
     uint32_t tau = 0u;
-    if (ntiles >= nsel)
-        tau = radix_kth<NTHR, TPT, true>(nt_own, [&](int k) { return tk[k]; }, nsel, sc, 2).lower;
+    if ((ncand + KPT - 1) / KPT >= nsel)
+        tau = radix_kth<NTHR, 1>(n_t > 0 ? 1 : 0, [&](int) { return kmax; }, nsel, sc, 2).lower;
 
-    // 3. survivors: pages >= tau, from the live tiles (maximum >= tau)
-    int nlive_own = 0;
+    // 2. survivors, compacted in index order
+    int cnt = 0;
 #pragma unroll
-    for (int k = 0; k < TPT; ++k) nlive_own += k < nt_own && tk[k] >= tau;
-    int nlive;
-    int lpos = block_excl_scan<NTHR>(nlive_own, sc, &nlive);
+    for (int k = 0; k < KPT; ++k) cnt += k < n_t && key[k] >= tau;
+    int nsurv;
+    int pos = block_excl_scan<NTHR>(cnt, sc, &nsurv);
+    auto emit_page = [&](int o, int page) { out[o] = page; };
+    if (nsurv <= surv_cap) {
+        uint32_t* skey = surv;
+        int32_t* sidx = reinterpret_cast<int32_t*>(surv + surv_cap);
 #pragma unroll
-    for (int k = 0; k < TPT; ++k)
-        if (k < nt_own && tk[k] >= tau) live_tile[lpos++] = t0 + k;
-    __syncthreads();
-    int nsurv = 0;
-    bool overflow = false;
-    for (int r0 = 0; r0 < nlive; r0 += NTHR * kLivePerThread) {  // uniform trip count
-        uint32_t v[kLivePerThread][kTile];
-        int c0[kLivePerThread];
-        int cnt = 0;
-#pragma unroll
-        for (int m = 0; m < kLivePerThread; ++m) {
-            const int li = r0 + tid * kLivePerThread + m;  // consecutive per thread
-            c0[m] = li < nlive ? live_tile[li] * kTile : ncand;
-#pragma unroll
-            for (int i = 0; i < kTile; ++i)
-                v[m][i] = c0[m] + i < ncand ? cand_key(c0[m] + i) : 0u;
-        }
-#pragma unroll
-        for (int m = 0; m < kLivePerThread; ++m)
-#pragma unroll
-            for (int i = 0; i < kTile; ++i) cnt += v[m][i] >= tau && v[m][i] != 0u;
-        int total;
-        int pos = nsurv + block_excl_scan<NTHR>(cnt, sc, &total);
-        if (nsurv + total > surv_cap) overflow = true;
-        if (!overflow) {
-#pragma unroll
-            for (int m = 0; m < kLivePerThread; ++m)
-#pragma unroll
-                for (int i = 0; i < kTile; ++i)
-                    if (v[m][i] >= tau && v[m][i] != 0u) {
-                        surv_key[pos] = v[m][i];
-                        surv_page[pos] = r.np + c0[m] + i;
-                        ++pos;
-                    }
-        }
-        nsurv += total;
-    }
-
-    if (!overflow) {
+        for (int k = 0; k < KPT; ++k)
+            if (k < n_t && key[k] >= tau) {
+                skey[pos] = key[k];
+                sidx[pos] = c0 + k;
+                ++pos;
+            }
         __syncthreads();
-        // 4. exact selection among the survivors (consecutive per thread)
+        // 3. exact selection among the survivors (consecutive per thread)
         const int per = (nsurv + NTHR - 1) / NTHR;
         const int base = tid * per;
-        const int n_t = max(0, min(per, nsurv - base));
-        auto key_at = [&](int k) { return surv_key[base + k]; };
-        const Kth t = radix_kth<NTHR, 0, false>(n_t, key_at, nsel, sc, 0);
-        write_selected<NTHR>(n_t, key_at, [&](int k) { return surv_page[base + k]; }, t.T,
-                             t.ties, sc, out);
+        const int m = max(0, min(per, nsurv - base));
+        auto skey_at = [&](int k) { return skey[base + k]; };
+        const Kth t = radix_kth<NTHR, 0>(m, skey_at, nsel, sc, 0);
+        write_selected<NTHR, 0>(m, skey_at, t.T, t.ties, sc,
+                                [&](int o, int k) { emit_page(o, r.np + sidx[base + k]); });
     } else {
-        // heavy ties: stream over every candidate, thread t owning a
-        // contiguous range, re-reading scores for each pass
-        const int per = (ncand + NTHR - 1) / NTHR;
-        const int base = tid * per;
-        const int n_t = max(0, min(per, ncand - base));
-        auto key_at = [&](int k) { return cand_key(base + k); };
-        const Kth t = radix_kth<NTHR, 0, false>(n_t, key_at, nsel, sc, 0);
-        write_selected<NTHR>(n_t, key_at, [&](int k) { return r.np + base + k; }, t.T, t.ties,
-                             sc, out);
+        // heavy ties: exact selection among every candidate
+        auto key_at = [&](int k) { return key[k]; };
+        const Kth t = radix_kth<NTHR, KPT>(n_t, key_at, nsel, sc, 0);
+        write_selected<NTHR, KPT>(n_t, key_at, t.T, t.ties, sc,
+                                  [&](int o, int k) { emit_page(o, r.np + c0 + k); });
     }
 }
 
