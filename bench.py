@@ -96,6 +96,26 @@ def algorithmic_bytes(lens, hq, hkv, D, prefix, window, budget, dense=False):
     return meta + kv + qo, meta, kv
 
 
+def stage_bytes(lens, hq, hkv, D, prefix, window, budget):
+    """Algorithmic bytes of the two HBM-bound stages of sparse_decode:
+    stage 1 reads the candidates' metadata, the prefix and window pages'
+    K and V, and q; stage 3 reads the selected pages' K and V and q."""
+    meta = forced = sel_kv = 0
+    for L in lens:
+        n, np_, ws = page_ranges(L, prefix, window)
+        nc = ws - np_
+        meta += nc * hkv * 4 * D
+        forced += (min(L, 16 * np_) + max(0, L - 16 * ws)) * hkv * 4 * D
+        sel_kv += 16 * min(budget, nc) * hkv * 4 * D
+    qb = len(lens) * hq * D * 2
+    return {1: meta + forced + qb, 3: sel_kv + qb}
+
+
+STAGES = {1: "score_forced", 2: "select", 3: "attend_selected", 4: "merge"}
+STAGE_KERNELS = {1: "score_forced_kernel", 2: "select_kernel", 3: "attend_kernel",
+                 4: "merge_kernel"}
+
+
 class Clocks:
     """Samples SM clock and clock-event reasons with NVML while running."""
 
@@ -172,10 +192,13 @@ def ncu_traffic():
         if len(parts) != 5 or not parts[2].isdigit():
             continue
         kernel, workload, nbytes, src, sha = parts
+        h = hashlib.sha1()
         try:
-            cur = hashlib.sha1(open(os.path.join(csrc, src), "rb").read()).hexdigest()[:12]
+            for f in src.split("+"):  # the kernel's files, concatenated in order
+                h.update(open(os.path.join(csrc, f), "rb").read())
         except OSError:
             continue
+        cur = h.hexdigest()[:12]
         if cur == sha:
             out[(kernel, workload)] = int(nbytes)
     return out
@@ -329,29 +352,31 @@ def run_ours(args, rank, world, local):
     peak, peak_kind = measured_peak()
     traffic = ncu_traffic()
 
-    # ---- per-kernel device times on the 64k state (standalone entry points)
+    # ---- per-kernel device times on the 64k state: each stage of
+    # sparse_decode launched alone (it re-reads what the earlier stages left)
     reps = args.reps
     stage(Wm + K - 1)
     sel64 = W64.sel[:, :, :x.budget]
-    kt = {}
-    kt["score_pages"] = timed(lambda: slc.score_pages(cur_q, W64.cache, W64.bt, cur_len, x.prefix,
-                                                       x.window, scores=W64.scores), reps, flush)
-    kt["select_pages"] = timed(lambda: slc.select_pages(W64.scores, cur_len, x.prefix, x.window,
-                                                         x.budget, selected=sel64), reps, flush)
-    kt["sparse_attend"] = timed(lambda: slc.sparse_attend(cur_q, W64.cache, W64.bt, cur_len,
-                                                          x.prefix, x.window, sel64, out=W64.out,
-                                                          workspace=W64.ws), reps, flush)
-    kt["kv_append"] = None  # measured inside the step only (its state changes)
-    _, meta64, kv64 = algorithmic_bytes([int(v) + Wm + K for v in L0], hq, hkv, D, x.prefix,
-                                        x.window, x.budget)
-    kbytes = {"score_pages": meta64 + B * hq * D * 2, "sparse_attend": kv64 + B * hq * D * 6}
-    dom = max(("score_pages", "sparse_attend"), key=lambda k: kt[k])
-    ach = kbytes[dom] / (kt[dom] * 1e-3) / 1e9
-    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": peak,
-                "unit": "GB/s", "frac": round(ach / peak, 4),
-                "traffic": traffic.get((dom, "decode64k")),
-                "algorithmic_bytes": kbytes[dom], "us_per_launch": round(kt[dom] * 1e3, 2),
-                "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind}
+    lens64 = [int(v) + Wm + K for v in L0]
+
+    def stage_times(w, q_, lens_t, xx):
+        slc.sparse_decode(q_, w.cache, w.bt, lens_t, xx.prefix, xx.window, xx.budget, out=w.out,
+                          workspace=w.ws)
+        return {k: timed(lambda k=k: slc.sparse_decode_stage(
+            k, q_, w.cache, w.bt, lens_t, xx.prefix, xx.window, xx.budget, out=w.out,
+            workspace=w.ws), reps, flush) for k in STAGES}
+
+    kt = stage_times(W64, cur_q, cur_len, x)
+    kb = stage_bytes(lens64, hq, hkv, D, x.prefix, x.window, x.budget)
+    dom = max((1, 3), key=lambda k: kt[k])  # the HBM-bound stages
+    ach = kb[dom] / (kt[dom] * 1e-3) / 1e9
+    roofline = {"kernel": STAGE_KERNELS[dom], "stage": STAGES[dom], "bound": "hbm",
+                "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(ach / peak, 4),
+                "traffic": traffic.get((STAGE_KERNELS[dom], "decode64k")),
+                "algorithmic_bytes": kb[dom], "us_per_launch": round(kt[dom] * 1e3, 2),
+                "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs, burst copy; the kernel is "
+                               "timed alone)" % peak_kind}
 
     # ---- dense comparison on the same 64k cache
     also = {}
@@ -366,7 +391,7 @@ def run_ours(args, rank, world, local):
             "sparse_us": round(sparse64 * 1e3, 2), "dense_us": round(dense64 * 1e3, 2),
             "speedup_vs_dense": round(dense64 / sparse64, 2),
             "dense_gbs": round(db / (dense64 * 1e-3) / 1e9, 1),
-            "kernel_us": {k: (round(v * 1e3, 2) if v else None) for k, v in kt.items()}}
+            "stage_us": {STAGES[k]: round(v * 1e3, 2) for k, v in kt.items()}}
 
     # ---- e2e through the public API: host buffers, copies inside the timing
     qh = torch.stack(qs).pin_memory()
@@ -416,19 +441,20 @@ def run_ours(args, rank, world, local):
         sp_graph = timed(gsp.replay, reps, flush)
         dn = timed(lambda: slc.dense_decode(W256.q, W256.cache, W256.bt, W256.sl, out=W256.out,
                                             workspace=W256.ws), max(5, reps // 4), flush)
-        sel256 = W256.sel[:, :, :y.budget]
-        k_score = timed(lambda: slc.score_pages(W256.q, W256.cache, W256.bt, W256.sl, y.prefix,
-                                                y.window, scores=W256.scores), reps, flush)
-        k_select = timed(lambda: slc.select_pages(W256.scores, W256.sl, y.prefix, y.window,
-                                                  y.budget, selected=sel256), reps, flush)
-        k_attend = timed(lambda: slc.sparse_attend(W256.q, W256.cache, W256.bt, W256.sl,
-                                                   y.prefix, y.window, sel256, out=W256.out,
-                                                   workspace=W256.ws), reps, flush)
+        kt256 = stage_times(W256, W256.q, W256.sl, y)
+        kb256 = stage_bytes(y.seq_lens.tolist(), y.wl.hq, y.wl.hkv, y.wl.head_dim, y.prefix,
+                            y.window, y.budget)
         db256, _, _ = algorithmic_bytes(y.seq_lens.tolist(), y.wl.hq, y.wl.hkv, y.wl.head_dim,
                                         0, 0, 0, True)
-        sb = b256[1] + y.wl.batch * y.wl.hq * y.wl.head_dim * 2
-        ab = b256[2] + y.wl.batch * y.wl.hq * y.wl.head_dim * 6
         best = min(sp, sp_graph)
+
+        def stage_entry(k):
+            e = {"kernel": STAGE_KERNELS[k], "us": round(kt256[k] * 1e3, 2)}
+            if k in kb256:
+                g = kb256[k] / (kt256[k] * 1e-3) / 1e9
+                e.update({"bytes": kb256[k], "gbs": round(g, 1), "frac": round(g / peak, 4),
+                          "traffic": traffic.get((STAGE_KERNELS[k], "decode256k"))})
+            return e
         also["decode256k"] = {
             "workload": "B=4, ctx 262144, Hq 32 / Hkv 4, d 128, page 16, prefix 128, "
                         "window 4096, budget 256 pages, 64 needles/seq",
@@ -439,16 +465,7 @@ def run_ours(args, rank, world, local):
             "hbm_gbs": round(b256[0] / (best * 1e-3) / 1e9, 1),
             "step_roofline_frac": round(b256[0] / (best * 1e-3) / 1e9 / peak, 4),
             "dense_gbs": round(db256 / (dn * 1e-3) / 1e9, 1),
-            "kernels": {
-                "score_pages": {"us": round(k_score * 1e3, 2), "bytes": sb,
-                                "gbs": round(sb / (k_score * 1e-3) / 1e9, 1),
-                                "frac": round(sb / (k_score * 1e-3) / 1e9 / peak, 4),
-                                "traffic": traffic.get(("score_pages", "decode256k"))},
-                "select_pages": {"us": round(k_select * 1e3, 2)},
-                "sparse_attend": {"us": round(k_attend * 1e3, 2), "bytes": ab,
-                                  "gbs": round(ab / (k_attend * 1e-3) / 1e9, 1),
-                                  "frac": round(ab / (k_attend * 1e-3) / 1e9 / peak, 4),
-                                  "traffic": traffic.get(("sparse_attend", "decode256k"))}}}
+            "stages": {STAGES[k]: stage_entry(k) for k in STAGES}}
         assert slc.device_status() == 0
 
     result = {
@@ -459,7 +476,8 @@ def run_ours(args, rank, world, local):
         "config": {
             "workload": "decode64k: B=4, ctx 65536 (+1 token per step), Hq 32 / Hkv 4, d 128, "
                         "page 16, prefix 128, window 1024, budget 128 pages, 64 needles/seq; "
-                        "step = kv_append + sparse_decode (score, select, attend, merge), "
+                        "step = kv_append + sparse_decode (score with prefix/window "
+                        "attention, select, selected attention, merge), "
                         "CUDA graph",
             "global_batch": B * world, "seq_len": int(L0[0]), "parallelism": "replicas",
             "l2": "flushed (256 MiB write) before every timed step, outside its events"},

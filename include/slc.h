@@ -150,6 +150,22 @@ SLC_API int slc_sparse_decode(const void *q, const slc_cache_t *cache, const int
                       float scale, float *out, int32_t *selected_out, void *workspace,
                       size_t workspace_bytes, slc_stream_t stream);
 
+/* One stage of slc_sparse_decode alone (same arguments), for timing and
+ * inspection; the stages run in this order and each reads what the earlier
+ * ones left in the workspace (and in selected_out):
+ *   1  score the candidate pages and attend the prefix and window pages
+ *   2  select the pages
+ *   3  attend the selected pages
+ *   4  merge the split partials into out
+ * Running 1, 2, 3, 4 in order equals one slc_sparse_decode call.  Returns
+ * SLC_ERR_INVALID_ARG for any other stage. */
+SLC_API int slc_sparse_decode_stage(int32_t stage, const void *q, const slc_cache_t *cache,
+                            const int32_t *block_table, int32_t max_pages_per_seq,
+                            const int32_t *seq_lens, int32_t batch, int32_t num_q_heads,
+                            int32_t prefix, int32_t window, int32_t budget, float scale,
+                            float *out, int32_t *selected_out, void *workspace,
+                            size_t workspace_bytes, slc_stream_t stream);
+
 /* Attention over the prefix pages, the window pages and a caller-given
  * selection (same layout as slc_select_pages writes: [batch][num_kv_heads]
  * [budget] ascending logical pages, -1 padded; entries must be candidate

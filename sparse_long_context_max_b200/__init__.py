@@ -33,7 +33,8 @@ PAGE = 16
 
 # kernels one call launches (sparse: score with forced attention, select, attend,
 # merge; dense and attend: attend, merge)
-KERNELS_PER_CALL = {"sparse_decode": 4, "dense_decode": 2, "sparse_attend": 2, "kv_append": 1,
+KERNELS_PER_CALL = {"sparse_decode": 4, "sparse_decode_stage": 1, "dense_decode": 2,
+                    "sparse_attend": 2, "kv_append": 1,
                     "build_page_meta": 1, "score_pages": 1, "select_pages": 1}
 
 STATUS_BITS = {1: "bad page", 2: "bad length", 4: "bad selection", 8: "wait timeout"}
@@ -68,6 +69,7 @@ def _load() -> ctypes.CDLL:
         "slc_sparse_decode": (I, [P, C, P, I, P, I, I, I, I, I, F, P, P, P, Z, P]),
         "slc_dense_decode": (I, [P, C, P, I, P, I, I, F, P, P, Z, P]),
         "slc_sparse_attend": (I, [P, C, P, I, P, I, I, I, I, I, P, F, P, P, Z, P]),
+        "slc_sparse_decode_stage": (I, [I, P, C, P, I, P, I, I, I, I, I, F, P, P, P, Z, P]),
         "slc_device_status": (I, [ctypes.POINTER(ctypes.c_int32), P]),
         "slc_error_string": (ctypes.c_char_p, [ctypes.c_int]),
         "slc_last_cuda_error": (ctypes.c_char_p, []),
@@ -221,6 +223,31 @@ def sparse_decode(q, cache: PagedCache, block_table, seq_lens, prefix, window, b
                                   hq, prefix, window, budget, float(scale), _ptr(out),
                                   _ptr(selected_out), _ptr(workspace), workspace.numel(),
                                   _stream()))
+    return out
+
+
+def sparse_decode_stage(stage, q, cache: PagedCache, block_table, seq_lens, prefix, window,
+                        budget, scale=0.0, out=None, selected_out=None, workspace=None):
+    """One stage (1 score + prefix/window attention, 2 select, 3 selected
+    attention, 4 merge) of sparse_decode alone; stages 1..4 in order equal
+    one sparse_decode call on the same workspace."""
+    _need(q, torch.bfloat16, "q", 3)
+    _need(block_table, torch.int32, "block_table", 2)
+    _need(seq_lens, torch.int32, "seq_lens", 1)
+    B, hq, d = q.shape
+    mp = block_table.shape[1]
+    if out is None:
+        out = torch.empty((B, hq, d), dtype=torch.float32, device=q.device)
+    _need(out, torch.float32, "out", 3)
+    if selected_out is not None:
+        _need(selected_out, torch.int32, "selected_out", 3)
+    need = workspace_size(B, hq, cache.num_kv_heads, d, mp, budget)
+    if workspace is None:
+        workspace = _workspace(q.device, need)
+    _check(_lib.slc_sparse_decode_stage(int(stage), _ptr(q), cache.c, _ptr(block_table), mp,
+                                        _ptr(seq_lens), B, hq, prefix, window, budget,
+                                        float(scale), _ptr(out), _ptr(selected_out),
+                                        _ptr(workspace), workspace.numel(), _stream()))
     return out
 
 

@@ -209,7 +209,7 @@ static int decode(int mode, const void* q, const slc_cache_t* cache,
                   const int32_t* seq_lens, int32_t batch, int32_t num_q_heads, int32_t prefix,
                   int32_t window, int32_t budget, float scale, float* out,
                   int32_t* selected_out, void* workspace, size_t workspace_bytes,
-                  cudaStream_t stream) {
+                  cudaStream_t stream, int stage = 0) {
     const bool sparse = mode != 0;
     int rc = check_cache(cache);
     if (rc) return rc;
@@ -265,7 +265,7 @@ static int decode(int mode, const void* q, const slc_cache_t* cache,
         fp.se = SelectParams{scores, seq_lens, sel,    dev->status, batch, hkv,
                              max_pages_per_seq, prefix, window, budget, cs};
         fp.at = ap;
-        e = launch_sparse_fused(fp, D, dev->num_sms, stream);
+        e = launch_sparse_fused(fp, D, dev->num_sms, stream, stage);
         return e == cudaSuccess ? SLC_OK : note_cuda(e, "sparse decode");
     }
     e = launch_attend(ap, D, dev->num_sms, stream, nullptr);
@@ -280,6 +280,18 @@ int slc_sparse_decode(const void* q, const slc_cache_t* cache, const int32_t* bl
     return decode(1, q, cache, block_table, max_pages_per_seq, seq_lens, batch, num_q_heads,
                   prefix, window, budget, scale, out, selected_out, workspace, workspace_bytes,
                   stream);
+}
+
+int slc_sparse_decode_stage(int32_t stage, const void* q, const slc_cache_t* cache,
+                            const int32_t* block_table, int32_t max_pages_per_seq,
+                            const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                            int32_t prefix, int32_t window, int32_t budget, float scale,
+                            float* out, int32_t* selected_out, void* workspace,
+                            size_t workspace_bytes, slc_stream_t stream) {
+    if (stage < 1 || stage > 4) return SLC_ERR_INVALID_ARG;
+    return decode(1, q, cache, block_table, max_pages_per_seq, seq_lens, batch, num_q_heads,
+                  prefix, window, budget, scale, out, selected_out, workspace, workspace_bytes,
+                  stream, stage);
 }
 
 int slc_sparse_attend(const void* q, const slc_cache_t* cache, const int32_t* block_table,

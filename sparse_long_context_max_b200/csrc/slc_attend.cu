@@ -176,8 +176,10 @@ constexpr int attend_smem() {
     return NW * STAGES * (2 * kPage * D * 2 + 8 + 4);
 }
 
+// CTAs (chunks) of an attention launch: all that fit on the GPU at once,
+// at most kMaxAttendChunks.
 template <int D, int NW, int STAGES>
-cudaError_t run(AttendParams& p, int num_sms, cudaStream_t stream, bool merge, int* launched) {
+cudaError_t grid_of(int num_sms, int* blocks) {
     constexpr int smem = attend_smem<D, NW, STAGES>();
     static int occ = 0;
     if (occ == 0) {
@@ -189,8 +191,17 @@ cudaError_t run(AttendParams& p, int num_sms, cudaStream_t stream, bool merge, i
         if (e != cudaSuccess) return e;
         if (occ < 1) occ = 1;
     }
-    int blocks = num_sms * occ;
-    if (blocks > kMaxAttendChunks) blocks = kMaxAttendChunks;
+    *blocks = num_sms * occ;
+    if (*blocks > kMaxAttendChunks) *blocks = kMaxAttendChunks;
+    return cudaSuccess;
+}
+
+template <int D, int NW, int STAGES>
+cudaError_t run(AttendParams& p, int num_sms, cudaStream_t stream, bool merge, int* launched) {
+    constexpr int smem = attend_smem<D, NW, STAGES>();
+    int blocks = 0;
+    cudaError_t e0 = grid_of<D, NW, STAGES>(num_sms, &blocks);
+    if (e0 != cudaSuccess) return e0;
     p.num_chunks = blocks;  // chunk count (one chunk per CTA)
     cudaError_t e = launch_pdl(attend_kernel<D, NW, STAGES>, dim3(blocks), dim3(NW * 32), smem,
                                stream, p);
@@ -217,6 +228,15 @@ cudaError_t launch_attend_partials(AttendParams& p, int head_dim, int num_sms,
     if (p.batch * p.hkv == 0) return cudaSuccess;
     if (head_dim == 128) return run<128, 4, 2>(p, num_sms, stream, false, nullptr);
     return run<256, 4, 3>(p, num_sms, stream, false, nullptr);
+}
+
+int attend_chunks(int head_dim, int num_sms) {
+    int blocks = 1;
+    if (head_dim == 128)
+        grid_of<128, 4, 2>(num_sms, &blocks);
+    else
+        grid_of<256, 4, 3>(num_sms, &blocks);
+    return blocks;
 }
 
 }  // namespace slc

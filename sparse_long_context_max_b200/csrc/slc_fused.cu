@@ -296,8 +296,9 @@ __global__ void __launch_bounds__(kMergeGroups * D / 4) merge_kernel(FusedParams
     }
 }
 
+// stage 0: the four kernels; 1..4: that kernel alone.
 template <int D>
-cudaError_t run_sparse(const FusedParams& p, int num_sms, cudaStream_t stream) {
+cudaError_t run_sparse(const FusedParams& p, int num_sms, cudaStream_t stream, int stage) {
     using F = FusedGeom<D>;
     static int occ = 0;
     if (occ == 0) {
@@ -313,28 +314,38 @@ cudaError_t run_sparse(const FusedParams& p, int num_sms, cudaStream_t stream) {
     const int grid = num_sms * occ;
     FusedParams q = p;
     q.forced_chunks = grid;  // about one chunk per CTA
-    cudaError_t e = launch_pdl(score_forced_kernel<D>, dim3(grid), dim3(F::NTHR), F::SMEM, stream,
-                               q);
+    cudaError_t e = cudaSuccess;
+    if (stage == 0 || stage == 1)
+        e = launch_pdl(score_forced_kernel<D>, dim3(grid), dim3(F::NTHR), F::SMEM, stream, q);
     if (e != cudaSuccess) return e;
     q.at.list = kListSelected;
     q.at.slot_base = (long long)U + kMaxAttendChunks;
     q.at.num_chunks = 1;
     if (p.se.budget > 0) {
-        e = launch_select(p.se, stream);
-        if (e == cudaSuccess) e = launch_attend_partials(q.at, D, num_sms, stream);
+        if (stage == 0 || stage == 2) e = launch_select(p.se, stream);
         if (e != cudaSuccess) return e;
+        // the attention launcher sets num_chunks, which the merge needs
+        AttendParams at = q.at;
+        if (stage == 0 || stage == 3)
+            e = launch_attend_partials(at, D, num_sms, stream);
+        else
+            at.num_chunks = attend_chunks(D, num_sms);
+        if (e != cudaSuccess) return e;
+        q.at.num_chunks = at.num_chunks;
     }
-    return launch_pdl(merge_kernel<D>, dim3(U, p.at.group), dim3(kMergeGroups * D / 4), 0, stream,
-                      q);
+    if (stage == 0 || stage == 4)
+        e = launch_pdl(merge_kernel<D>, dim3(U, p.at.group), dim3(kMergeGroups * D / 4), 0, stream,
+                       q);
+    return e;
 }
 
 }  // namespace
 
 cudaError_t launch_sparse_fused(const FusedParams& p, int head_dim, int num_sms,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, int stage) {
     if (p.sc.batch * p.sc.hkv == 0) return cudaSuccess;
-    if (head_dim == 128) return run_sparse<128>(p, num_sms, stream);
-    return run_sparse<256>(p, num_sms, stream);
+    if (head_dim == 128) return run_sparse<128>(p, num_sms, stream, stage);
+    return run_sparse<256>(p, num_sms, stream, stage);
 }
 
 }  // namespace slc

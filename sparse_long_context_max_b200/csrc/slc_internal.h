@@ -128,7 +128,7 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
 // sparse_decode's path: four kernels chained by programmatic dependent
 // launch (score + forced attention, select, selected attention, merge).
 cudaError_t launch_sparse_fused(const FusedParams& p, int head_dim, int num_sms,
-                                cudaStream_t stream);
+                                cudaStream_t stream, int stage = 0);
 // Attention over the list of each unit (dense: all pages; sparse: prefix,
 // selected, window), then the merge of the per-warp partials into out.
 cudaError_t launch_attend(AttendParams p, int head_dim, int num_sms, cudaStream_t stream,
@@ -137,5 +137,7 @@ cudaError_t launch_attend(AttendParams p, int head_dim, int num_sms, cudaStream_
 // p.num_chunks (at most kMaxAttendChunks).
 cudaError_t launch_attend_partials(AttendParams& p, int head_dim, int num_sms,
                                    cudaStream_t stream);
+// The chunk count launch_attend_partials uses.
+int attend_chunks(int head_dim, int num_sms);
 
 }  // namespace slc

@@ -112,6 +112,12 @@ def test_decode_argument_validation():
     assert lib.slc_score_pages(FAKE, ctypes.byref(c), FAKE, 10, FAKE, 1, 8, -1, 0, FAKE,
                                None) == INVALID
     assert lib.slc_device_status(None, None) == INVALID
+    for stage in (0, 5, -1):  # only stages 1..4 exist
+        assert lib.slc_sparse_decode_stage(stage, FAKE, ctypes.byref(c), FAKE, 10, FAKE, 1, 8, 0,
+                                           0, 2, 0.0, FAKE, None, FAKE, 1 << 40,
+                                           None) == INVALID
+    assert lib.slc_sparse_decode_stage(2, FAKE, ctypes.byref(c), FAKE, 10, FAKE, 1, 7, 0, 0, 2,
+                                       0.0, FAKE, None, FAKE, 1 << 40, None) == INVALID  # Hq % Hkv
 
 
 def test_binding_rejects_cpu_tensors():

@@ -137,6 +137,35 @@ def test_tiny_sparse_parity(tiny):
     check_output(x, out, x.prefix, x.window, sel)
 
 
+def test_stages_in_order_equal_one_call():
+    """slc_sparse_decode_stage 1..4 on one workspace reproduce slc_sparse_decode
+    bit for bit (same kernels, same order)."""
+    import sparse_long_context_max_b200 as slc
+    x = synth.make_inputs(W["ragged"])
+    d = Dev(x)
+    B, hq, D = x.q.shape
+    hkv = x.k_cache.shape[1]
+    ws = torch.zeros(slc.workspace_size(B, hq, hkv, D, x.block_table.shape[1], x.budget),
+                     dtype=torch.uint8, device="cuda")
+    sel1 = torch.empty((B, hkv, x.budget), dtype=torch.int32, device="cuda")
+    sel2 = torch.full_like(sel1, -7)
+    out1 = slc.sparse_decode(d.q, d.cache, d.bt, d.sl, x.prefix, x.window, x.budget,
+                             selected_out=sel1, workspace=ws)
+    out2 = torch.full_like(out1, float("nan"))
+    ws.zero_()
+    for stage in (1, 2, 3, 4):
+        slc.sparse_decode_stage(stage, d.q, d.cache, d.bt, d.sl, x.prefix, x.window, x.budget,
+                                out=out2, selected_out=sel2, workspace=ws)
+    torch.cuda.synchronize()
+    assert slc.device_status() == 0
+    assert torch.equal(sel1, sel2)
+    assert torch.equal(out1, out2)
+    for bad in (0, 5, -1):
+        with pytest.raises(slc.SLCError):
+            slc.sparse_decode_stage(bad, d.q, d.cache, d.bt, d.sl, x.prefix, x.window, x.budget,
+                                    out=out2, selected_out=sel2, workspace=ws)
+
+
 def test_tiny_dense_parity(tiny):
     check_output(tiny.x, tiny.dense(), 0, 0, None, dense=True)
 
