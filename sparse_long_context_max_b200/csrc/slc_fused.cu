@@ -11,14 +11,18 @@
 //      rides along with the scoring, and the scores are written last, so
 //      the selection finds them in L2.
 //   2. select_kernel (slc_select.cu): one CTA per unit, from the scores the
-//      first kernel left.
+//      first kernel left; one more CTA per unit merges its forced-chunk
+//      partials.
 //   3. attend_kernel (slc_attend.cu) over the selected pages of all units.
 //   4. merge_kernel: log-sum-exp merge of both kernels' partials per (unit,
 //      query head).
 //
 // Partials: forced chunk c of unit u goes to slot u + c, selected chunk c
 // to slot U + kMaxAttendChunks + u + c (U units); a chunk covers
-// consecutive list positions, so each slot is written once.
+// consecutive list positions, so each slot is written once.  Extra CTAs of
+// the selection kernel merge each unit's forced-chunk partials into slot
+// 2 (U + kMaxAttendChunks) + u while the selection runs, so the final merge
+// combines that one slot with the selected-chunk slots.
 #include "slc_attend_impl.cuh"
 #include "slc_score_impl.cuh"
 
@@ -60,23 +64,6 @@ __device__ __forceinline__ int unit_tiles(const ScoreParams& p, int budget, int 
     const PageRanges r = page_ranges(L, p.prefix, p.window);
     const int ncand = r.ws - r.np;
     return ncand > budget ? (ncand + scr::kTilePages - 1) / scr::kTilePages : 0;
-}
-
-// Chunking of the forced lists into about `target` chunks: total positions,
-// chunk count, positions per chunk.  Warp-wide; the scoring and merge
-// kernels compute it identically.
-struct Chunking {
-    long long total, chunks, cpp;
-};
-__device__ __forceinline__ Chunking forced_chunking(const AttendParams& at, int target) {
-    auto len_of = [&](int b) { return attn::list_len(at, b); };
-    Chunking c;
-    c.total = total_units(at.batch, at.hkv, len_of);
-    long long n = c.total < target ? c.total : target;
-    if (n > kMaxAttendChunks) n = kMaxAttendChunks;
-    c.cpp = n > 0 ? (c.total + n - 1) / n : 1;
-    c.chunks = n > 0 ? (c.total + c.cpp - 1) / c.cpp : 0;
-    return c;
 }
 
 __device__ __forceinline__ AttendParams with_list(const AttendParams& at, int list) {
@@ -183,7 +170,7 @@ __global__ void __launch_bounds__(FusedGeom<D>::NTHR, FusedGeom<D>::MINB)
     grid_dep_launch();
 
     const AttendParams atF = with_list(p.at, kListForced);
-    const Chunking cf = forced_chunking(atF, p.forced_chunks);
+    const attn::Chunking cf = attn::forced_chunking(atF, p.forced_chunks);
     uint32_t it = 0;
     bool ok = true;
     for (long long c = blockIdx.x; c < cf.chunks; c += gridDim.x) {
@@ -224,7 +211,7 @@ __global__ void __launch_bounds__(kMergeGroups * D / 4) merge_kernel(FusedParams
     __shared__ float4 sh_num[kMergeGroups][V4];
     __shared__ float sh_den[kMergeGroups];
     if (tid < 32) {
-        const Chunking cf = forced_chunking(atF, p.forced_chunks);
+        const attn::Chunking cf = attn::forced_chunking(atF, p.forced_chunks);
         auto len_sel = [&](int bb) { return attn::list_len(atS, bb); };
         const long long totalS = total_units(atS.batch, atS.hkv, len_sel);
         const long long cppS = totalS > 0 ? (totalS + p.at.num_chunks - 1) / p.at.num_chunks : 1;
@@ -232,8 +219,11 @@ __global__ void __launch_bounds__(kMergeGroups * D / 4) merge_kernel(FusedParams
         const long long sB = attn::unit_list_start(atS, u);
         const int lenA = attn::list_len(atF, b), lenB = attn::list_len(atS, b);
         if (tid == 0) {
-            sh_r[0] = lenA > 0 ? u + sA / cf.cpp : 0;
-            sh_r[1] = lenA > 0 ? u + (sA + lenA - 1) / cf.cpp : -1;
+            // the forced-list partials, merged into one slot by the selection
+            // kernel when it ran
+            const bool pre = p.premerged_base >= 0;
+            sh_r[0] = lenA > 0 ? (pre ? p.premerged_base + u : u + sA / cf.cpp) : 0;
+            sh_r[1] = lenA > 0 ? (pre ? p.premerged_base + u : u + (sA + lenA - 1) / cf.cpp) : -1;
             sh_r[2] = lenB > 0 ? p.at.slot_base + u + sB / cppS : 0;
             sh_r[3] = lenB > 0 ? p.at.slot_base + u + (sB + lenB - 1) / cppS : -1;
         }
@@ -321,8 +311,16 @@ cudaError_t run_sparse(const FusedParams& p, int num_sms, cudaStream_t stream, i
     q.at.list = kListSelected;
     q.at.slot_base = (long long)U + kMaxAttendChunks;
     q.at.num_chunks = 1;
+    q.premerged_base = -1;
     if (p.se.budget > 0) {
-        if (stage == 0 || stage == 2) e = launch_select(p.se, stream);
+        PremergeParams pm;
+        pm.at = p.at;
+        pm.at.list = kListForced;
+        pm.forced_chunks = grid;
+        pm.dst_base = 2 * ((long long)U + kMaxAttendChunks);
+        pm.v4 = D / 4;
+        q.premerged_base = pm.dst_base;
+        if (stage == 0 || stage == 2) e = launch_select(p.se, stream, &pm);
         if (e != cudaSuccess) return e;
         // the attention launcher sets num_chunks, which the merge needs
         AttendParams at = q.at;

@@ -113,10 +113,19 @@ struct FusedParams {
     SelectParams se;
     AttendParams at;  // list is set per kernel
     int forced_chunks;  // target chunk count of the prefix/window attention
+    long long premerged_base;  // >= 0: unit u's forced partials merged into this + u
+};
+// Merge of every unit's forced-list partials into one slot per unit, done
+// by extra CTAs of the selection kernel.
+struct PremergeParams {
+    AttendParams at;    // the forced lists
+    int forced_chunks;  // as FusedParams::forced_chunks
+    long long dst_base;
+    int v4;  // head_dim / 4
 };
 // Split-partial slots of the sparse decode: two attention launches of at
-// most units + kMaxAttendChunks slots each.
-inline size_t fused_slots(size_t units) { return 2 * (units + kMaxAttendChunks); }
+// most units + kMaxAttendChunks slots each, then one merged slot per unit.
+inline size_t fused_slots(size_t units) { return 2 * (units + kMaxAttendChunks) + units; }
 WorkspaceLayout workspace_layout(int batch, int hq, int hkv, int head_dim, int max_pages,
                                  int budget);
 
@@ -124,7 +133,10 @@ cudaError_t launch_kv_append(const KvAppendParams& p, int head_dim, cudaStream_t
 cudaError_t launch_build_meta(const BuildMetaParams& p, int head_dim, int num_sms,
                               cudaStream_t stream);
 cudaError_t launch_score(const ScoreParams& p, int head_dim, int num_sms, cudaStream_t stream);
-cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
+// The selection; with pm, extra CTAs also merge each unit's forced-list
+// partials (they run beside the selection CTAs).
+cudaError_t launch_select(const SelectParams& p, cudaStream_t stream,
+                          const PremergeParams* pm = nullptr);
 // sparse_decode's path: four kernels chained by programmatic dependent
 // launch (score + forced attention, select, selected attention, merge).
 cudaError_t launch_sparse_fused(const FusedParams& p, int head_dim, int num_sms,

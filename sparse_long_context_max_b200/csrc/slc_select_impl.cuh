@@ -242,14 +242,33 @@ __device__ void write_selected(int n_t, KeyAt key_at, uint32_t T, int ties, Scra
 }
 
 // Select the pages of unit u (all NTHR threads of the CTA call it; the
-// unit's candidates must number at most NTHR * KPT).  surv is shared memory
-// for surv_cap survivors (keys, then candidate indices).
+// unit's candidates must number at most NTHR * KPT, and a candidate-indexed
+// row at most NTHR * KPT floats).  surv is shared memory for surv_cap
+// survivors (keys, then candidate indices); stage holds the score row and
+// bar is an mbarrier in shared memory.
 template <int NTHR, int KPT>
 __device__ void select_unit(const SelectParams& p, int u, Scratch<NTHR>& sc, uint32_t* surv,
                             int surv_cap, float* stage, uint64_t* bar) {
     static_assert(KPT % 4 == 0, "16-byte loads");
     const int b = u / p.hkv;
     const int tid = threadIdx.x;
+    // rows by candidate (16-byte aligned, padded, at most NTHR * KPT floats):
+    // one bulk copy (TMA engine) of the whole row into `stage`, issued before
+    // the lengths are read -- a single CTA cannot keep that many plain loads
+    // in flight
+    const bool bulk = p.cand_stride > 0;
+    if (bulk && tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        const uint32_t bytes = (uint32_t)p.cand_stride * 4;
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_g2s(stage, p.scores + (long long)u * p.cand_stride, bytes, bar);
+    }
+    auto landed = [&]() {  // every thread; the copy must land before the CTA exits
+        __syncthreads();     // the barrier is initialised
+        if (!mbar_wait_bounded(bar, 0, 1u << 22) && tid == 0)
+            atomicOr(p.status, SLC_STATUS_WAIT_TIMEOUT);
+    };
     const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
     const PageRanges r = page_ranges(L, p.prefix, p.window);
     const int ncand = r.ws - r.np;
@@ -258,29 +277,21 @@ __device__ void select_unit(const SelectParams& p, int u, Scratch<NTHR>& sc, uin
 
     if (nsel >= ncand) {  // every candidate is kept (also covers ncand == 0)
         for (int i = tid; i < p.budget; i += NTHR) out[i] = i < ncand ? r.np + i : -1;
+        if (bulk) landed();
         return;
     }
     for (int i = nsel + tid; i < p.budget; i += NTHR) out[i] = -1;
-    if (nsel <= 0) return;
+    if (nsel <= 0) {
+        if (bulk) landed();
+        return;
+    }
 
     // candidate c's score: rows by candidate (16-byte aligned), or by page
     const int c0 = tid * KPT;
     const int n_t = max(0, min(KPT, ncand - c0));
     float f[KPT];
-    if (p.cand_stride) {
-        // one bulk copy (TMA engine) of the unit's row into `stage`: a single
-        // CTA cannot keep that many plain loads in flight
-        if (tid == 0) {
-            mbar_init(bar, 1);
-            fence_mbar_init();
-            const uint32_t bytes = (uint32_t)((ncand + 3) / 4) * 16;  // rows are padded
-            mbar_arrive_expect_tx(bar, bytes);
-            bulk_g2s(stage, p.scores + (long long)u * p.cand_stride, bytes, bar);
-        }
-        __syncthreads();  // the barrier is initialised
-        if (!mbar_wait_bounded(bar, 0, 1u << 22)) {
-            if (tid == 0) atomicOr(p.status, SLC_STATUS_WAIT_TIMEOUT);
-        }
+    if (bulk) {
+        landed();
         const float4* s4 = reinterpret_cast<const float4*>(stage + c0);
 #pragma unroll
         for (int q = 0; q < KPT / 4; ++q) {
