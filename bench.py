@@ -98,22 +98,20 @@ def algorithmic_bytes(lens, hq, hkv, D, prefix, window, budget, dense=False):
 
 def stage_bytes(lens, hq, hkv, D, prefix, window, budget):
     """Algorithmic bytes of the two HBM-bound stages of sparse_decode:
-    stage 1 reads the candidates' metadata, the prefix and window pages'
-    K and V, and q; stage 3 reads the selected pages' K and V and q."""
-    meta = forced = sel_kv = 0
+    stage 1 reads the candidates' metadata and q; stage 3 reads the K and V
+    of the prefix, window and selected pages and q."""
+    meta = kv = 0
     for L in lens:
         n, np_, ws = page_ranges(L, prefix, window)
         nc = ws - np_
         meta += nc * hkv * 4 * D
-        forced += (min(L, 16 * np_) + max(0, L - 16 * ws)) * hkv * 4 * D
-        sel_kv += 16 * min(budget, nc) * hkv * 4 * D
+        kv += (min(L, 16 * np_) + max(0, L - 16 * ws) + 16 * min(budget, nc)) * hkv * 4 * D
     qb = len(lens) * hq * D * 2
-    return {1: meta + forced + qb, 3: sel_kv + qb}
+    return {1: meta + qb, 3: kv + qb}
 
 
-STAGES = {1: "score_forced", 2: "select", 3: "attend_selected", 4: "merge"}
-STAGE_KERNELS = {1: "score_forced_kernel", 2: "select_kernel", 3: "attend_kernel",
-                 4: "merge_kernel"}
+STAGES = {1: "score", 2: "select", 3: "attend", 4: "merge"}
+STAGE_KERNELS = {1: "score_kernel", 2: "select_kernel", 3: "attend_kernel", 4: "merge_kernel"}
 
 
 class Clocks:
@@ -368,7 +366,7 @@ def run_ours(args, rank, world, local):
 
     kt = stage_times(W64, cur_q, cur_len, x)
     kb = stage_bytes(lens64, hq, hkv, D, x.prefix, x.window, x.budget)
-    dom = max((1, 3), key=lambda k: kt[k])  # the HBM-bound stages
+    dom = max((1, 3), key=lambda k: kt[k])  # the slower HBM-bound stage
     ach = kb[dom] / (kt[dom] * 1e-3) / 1e9
     roofline = {"kernel": STAGE_KERNELS[dom], "stage": STAGES[dom], "bound": "hbm",
                 "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
@@ -476,8 +474,7 @@ def run_ours(args, rank, world, local):
         "config": {
             "workload": "decode64k: B=4, ctx 65536 (+1 token per step), Hq 32 / Hkv 4, d 128, "
                         "page 16, prefix 128, window 1024, budget 128 pages, 64 needles/seq; "
-                        "step = kv_append + sparse_decode (score with prefix/window "
-                        "attention, select, selected attention, merge), "
+                        "step = kv_append + sparse_decode (score, select, attend, merge), "
                         "CUDA graph",
             "global_batch": B * world, "seq_len": int(L0[0]), "parallelism": "replicas",
             "l2": "flushed (256 MiB write) before every timed step, outside its events"},

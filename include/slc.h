@@ -153,9 +153,9 @@ SLC_API int slc_sparse_decode(const void *q, const slc_cache_t *cache, const int
 /* One stage of slc_sparse_decode alone (same arguments), for timing and
  * inspection; the stages run in this order and each reads what the earlier
  * ones left in the workspace (and in selected_out):
- *   1  score the candidate pages and attend the prefix and window pages
+ *   1  score the candidate pages
  *   2  select the pages
- *   3  attend the selected pages
+ *   3  attend the prefix, window and selected pages
  *   4  merge the split partials into out
  * Running 1, 2, 3, 4 in order equals one slc_sparse_decode call.  Returns
  * SLC_ERR_INVALID_ARG for any other stage. */

@@ -84,7 +84,7 @@ WorkspaceLayout workspace_layout(int batch, int hq, int hkv, int head_dim, int m
     WorkspaceLayout w{};
     const size_t units = (size_t)batch * hkv;
     const size_t group = (size_t)(hq / hkv);
-    const size_t slots = fused_slots(units);
+    const size_t slots = partial_slots(units);
     size_t off = 0;
     w.scores = off;  // by candidate, in rows of cand_stride_of(max_pages)
     off = round_up(off + units * (size_t)cand_stride_of(max_pages) * sizeof(float), 256);
@@ -254,21 +254,29 @@ static int decode(int mode, const void* q, const slc_cache_t* cache,
     ap.window = window;
     ap.budget = sparse ? budget : 0;
     ap.scale_log2 = scale * 1.4426950408889634f;
-    if (mode == 1) {
+    if (mode == 1 && budget > 0) {
+        // score -> select; the attention then waits for the selection
         float* scores = reinterpret_cast<float*>(ws + w.scores);
         const int cs = cand_stride_of(max_pages_per_seq);
-        FusedParams fp{};
-        fp.sc = ScoreParams{q,           cache->meta, block_table, seq_lens,
-                            scores,      dev->status, batch,
-                            num_q_heads, hkv,         num_q_heads / hkv, max_pages_per_seq,
-                            cache->num_pages, prefix, window, cs};
-        fp.se = SelectParams{scores, seq_lens, sel,    dev->status, batch, hkv,
-                             max_pages_per_seq, prefix, window, budget, cs};
-        fp.at = ap;
-        e = launch_sparse_fused(fp, D, dev->num_sms, stream, stage);
-        return e == cudaSuccess ? SLC_OK : note_cuda(e, "sparse decode");
+        ScoreParams sp{q,           cache->meta, block_table, seq_lens,
+                       scores,      dev->status, batch,
+                       num_q_heads, hkv,         num_q_heads / hkv, max_pages_per_seq,
+                       cache->num_pages, prefix, window, cs};
+        SelectParams lp{scores, seq_lens, sel,    dev->status, batch, hkv,
+                        max_pages_per_seq, prefix, window, budget, cs};
+        if (stage == 0 || stage == 1) {
+            e = launch_score(sp, D, dev->num_sms, stream);
+            if (e != cudaSuccess) return note_cuda(e, "score_pages");
+        }
+        if (stage == 0 || stage == 2) {
+            e = launch_select(lp, stream);
+            if (e != cudaSuccess) return note_cuda(e, "select_pages");
+        }
+        ap.wait_first = 1;
     }
-    e = launch_attend(ap, D, dev->num_sms, stream, nullptr);
+    const int what = stage == 3 ? kAttendOnly : stage == 4 ? kMergeOnly : kAttendAndMerge;
+    if (stage == 1 || stage == 2) return SLC_OK;
+    e = launch_attend(ap, D, dev->num_sms, stream, what);
     return e == cudaSuccess ? SLC_OK : note_cuda(e, "attend/merge");
 }
 

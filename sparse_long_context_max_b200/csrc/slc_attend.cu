@@ -60,6 +60,9 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttendParams p) {
     }
     __syncwarp();
     grid_dep_launch();  // the merge may start; it waits before reading partials
+    // after a selection kernel, stream nothing before it is done: its
+    // latency-bound work runs without competing traffic
+    if (p.wait_first) grid_dep_wait();
 
     auto len_of = [&](int b) { return list_len(p, b); };
     const long long total = total_units(p.batch, p.hkv, len_of);
@@ -68,8 +71,7 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttendParams p) {
     const long long e = min(total, s + cpp);
     uint32_t it = 0;
     bool ok = true;
-    attend_range<D, NW, STAGES>(p, smem, ring, it, ok, s, e, blockIdx.x, p.slot_base,
-                                [](int) {});
+    attend_range<D, NW, STAGES>(p, smem, ring, it, ok, s, e, blockIdx.x, 0, [](int) {});
 }
 
 // Merge of the CTA partials of one (unit, query head): slots unit + chunk
@@ -197,46 +199,28 @@ cudaError_t grid_of(int num_sms, int* blocks) {
 }
 
 template <int D, int NW, int STAGES>
-cudaError_t run(AttendParams& p, int num_sms, cudaStream_t stream, bool merge, int* launched) {
+cudaError_t run(AttendParams p, int num_sms, cudaStream_t stream, int what) {
     constexpr int smem = attend_smem<D, NW, STAGES>();
     int blocks = 0;
-    cudaError_t e0 = grid_of<D, NW, STAGES>(num_sms, &blocks);
-    if (e0 != cudaSuccess) return e0;
+    cudaError_t e = grid_of<D, NW, STAGES>(num_sms, &blocks);
+    if (e != cudaSuccess) return e;
     p.num_chunks = blocks;  // chunk count (one chunk per CTA)
-    cudaError_t e = launch_pdl(attend_kernel<D, NW, STAGES>, dim3(blocks), dim3(NW * 32), smem,
-                               stream, p);
-    if (e != cudaSuccess || !merge) return e;
-    e = launch_pdl(merge_kernel<D>, dim3(p.batch * p.hkv, p.group), dim3(kMergeGroups * D / 4), 0,
-                   stream, p);
-    if (launched) *launched += 2;
-    return e;
+    if (what != kMergeOnly)
+        e = launch_pdl(attend_kernel<D, NW, STAGES>, dim3(blocks), dim3(NW * 32), smem, stream,
+                       p);
+    if (e != cudaSuccess || what == kAttendOnly) return e;
+    return launch_pdl(merge_kernel<D>, dim3(p.batch * p.hkv, p.group),
+                      dim3(kMergeGroups * D / 4), 0, stream, p);
 }
 
 }  // namespace
 
 cudaError_t launch_attend(AttendParams p, int head_dim, int num_sms, cudaStream_t stream,
-                          int* launched) {
+                          int what) {
     if (p.batch * p.hkv == 0) return cudaSuccess;
-    p.slot_base = 0;
     // D=128: 4 warps x 2 stages x 8 KB = 64 KB per CTA, three CTAs per SM
-    if (head_dim == 128) return run<128, 4, 2>(p, num_sms, stream, true, launched);
-    return run<256, 4, 3>(p, num_sms, stream, true, launched);
-}
-
-cudaError_t launch_attend_partials(AttendParams& p, int head_dim, int num_sms,
-                                   cudaStream_t stream) {
-    if (p.batch * p.hkv == 0) return cudaSuccess;
-    if (head_dim == 128) return run<128, 4, 2>(p, num_sms, stream, false, nullptr);
-    return run<256, 4, 3>(p, num_sms, stream, false, nullptr);
-}
-
-int attend_chunks(int head_dim, int num_sms) {
-    int blocks = 1;
-    if (head_dim == 128)
-        grid_of<128, 4, 2>(num_sms, &blocks);
-    else
-        grid_of<256, 4, 3>(num_sms, &blocks);
-    return blocks;
+    if (head_dim == 128) return run<128, 4, 2>(p, num_sms, stream, what);
+    return run<256, 4, 3>(p, num_sms, stream, what);
 }
 
 }  // namespace slc

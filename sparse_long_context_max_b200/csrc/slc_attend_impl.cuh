@@ -1,5 +1,5 @@
-// Split-KV flash-decode building blocks shared by the attention kernels
-// (slc_attend.cu) and the fused sparse decode (slc_fused.cu): page lists,
+// Split-KV flash-decode building blocks of the attention kernels
+// (slc_attend.cu): page lists,
 // the per-warp streaming attention over a list, the combine of a CTA's warp
 // partials into one split partial, and the log-sum-exp merge of a unit's
 // split partials.  slc_attend.cu describes the data flow and the
@@ -395,89 +395,6 @@ __device__ __forceinline__ long long unit_list_start(const AttendParams& p, int 
         base += c;
     }
     return base + (long long)h * list_len(p, b);
-}
-
-// Chunking of a unit-list kind into about `target` chunks: total positions,
-// chunk count, positions per chunk.  Warp-wide; every kernel that reads the
-// chunks' partials computes it identically.
-struct Chunking {
-    long long total, chunks, cpp;
-};
-__device__ __forceinline__ Chunking forced_chunking(const AttendParams& at, int target) {
-    auto len_of = [&](int b) { return list_len(at, b); };
-    Chunking c;
-    c.total = total_units(at.batch, at.hkv, len_of);
-    long long n = c.total < target ? c.total : target;
-    if (n > kMaxAttendChunks) n = kMaxAttendChunks;
-    c.cpp = n > 0 ? (c.total + n - 1) / n : 1;
-    c.chunks = n > 0 ? (c.total + c.cpp - 1) / c.cpp : 0;
-    return c;
-}
-
-// Log-sum-exp merge of one unit's partials in slots [a0, a1] into slot dst
-// (all NTHR threads of the CTA; V4 = head_dim / 4, G * V4 <= NTHR).
-// Threads split into slot groups x (query head, 4 dims); each group folds
-// its slots with online rescaling, then the groups combine through shared
-// memory (scratch: NTHR float4 + 2 * NTHR floats).
-template <int NTHR>
-__device__ void merge_slots(const AttendParams& p, int V4, long long a0, long long a1,
-                            long long dst, float4* sh_num, float* sh_m, float* sh_den) {
-    const int G = p.group;
-    const int pairs = G * V4;
-    const int groups = NTHR / pairs;  // >= 1
-    const int tid = threadIdx.x;
-    const int grp = tid / pairs, pr = tid % pairs;
-    const int g = pr / V4, d4 = pr % V4;
-    const int D = 4 * V4;
-    float M = -INFINITY, den = 0.f;
-    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (grp < groups) {
-#pragma unroll 4
-        for (long long k = a0 + grp; k <= a1; k += groups) {
-            const float2 ml = __ldcg(&p.part_ml[k * G + g]);
-            const float4 a =
-                __ldcg(reinterpret_cast<const float4*>(p.part_acc + (k * G + g) * D) + d4);
-            if (ml.x > M) {
-                const float c = ex2(M - ml.x);
-                num.x *= c;
-                num.y *= c;
-                num.z *= c;
-                num.w *= c;
-                den *= c;
-                M = ml.x;
-            }
-            const float w = ml.x == -INFINITY ? 0.f : ex2(ml.x - M);
-            num.x = fmaf(w, a.x, num.x);
-            num.y = fmaf(w, a.y, num.y);
-            num.z = fmaf(w, a.z, num.z);
-            num.w = fmaf(w, a.w, num.w);
-            den = fmaf(w, ml.y, den);
-        }
-        sh_num[tid] = num;
-        sh_m[tid] = M;
-        sh_den[tid] = den;
-    }
-    __syncthreads();
-    if (grp == 0) {
-        float Mt = -INFINITY;
-        for (int i = 0; i < groups; ++i) Mt = fmaxf(Mt, sh_m[i * pairs + pr]);
-        const float Mu = Mt == -INFINITY ? 0.f : Mt;
-        float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
-        float dt = 0.f;
-        for (int i = 0; i < groups; ++i) {
-            const float c = ex2(sh_m[i * pairs + pr] - Mu);  // 0 for an empty group
-            const float4 o = sh_num[i * pairs + pr];
-            tot.x = fmaf(c, o.x, tot.x);
-            tot.y = fmaf(c, o.y, tot.y);
-            tot.z = fmaf(c, o.z, tot.z);
-            tot.w = fmaf(c, o.w, tot.w);
-            dt = fmaf(c, sh_den[i * pairs + pr], dt);
-        }
-        // the merged partial keeps (max, sum) relative to Mt
-        reinterpret_cast<float4*>(p.part_acc + (dst * G + g) * D)[d4] = tot;
-        if (d4 == 0) p.part_ml[dst * G + g] = make_float2(Mt, dt);
-    }
-    __syncthreads();
 }
 
 }  // namespace attn

@@ -98,7 +98,7 @@ struct AttendParams {
     int prefix, window, budget;
     float scale_log2;  // softmax scale * log2(e)
     int num_chunks;    // chunks of the attention launch (one per CTA)
-    long long slot_base;  // this launch's partials: slot slot_base + unit + chunk
+    int wait_first;    // wait for the preceding kernel before any read (it wrote the selection)
 };
 
 // Workspace carve-up shared by the API and the size query.
@@ -106,50 +106,20 @@ struct WorkspaceLayout {
     size_t scores, selected, part_acc, part_ml, total;
 };
 
-// Sparse decode step (slc_fused.cu): scoring with the prefix/window
-// attention in one grid, selection, selected-page attention, merge.
-struct FusedParams {
-    ScoreParams sc;
-    SelectParams se;
-    AttendParams at;  // list is set per kernel
-    int forced_chunks;  // target chunk count of the prefix/window attention
-    long long premerged_base;  // >= 0: unit u's forced partials merged into this + u
-};
-// Merge of every unit's forced-list partials into one slot per unit, done
-// by extra CTAs of the selection kernel.
-struct PremergeParams {
-    AttendParams at;    // the forced lists
-    int forced_chunks;  // as FusedParams::forced_chunks
-    long long dst_base;
-    int v4;  // head_dim / 4
-};
-// Split-partial slots of the sparse decode: two attention launches of at
-// most units + kMaxAttendChunks slots each, then one merged slot per unit.
-inline size_t fused_slots(size_t units) { return 2 * (units + kMaxAttendChunks) + units; }
-WorkspaceLayout workspace_layout(int batch, int hq, int hkv, int head_dim, int max_pages,
-                                 int budget);
+// Split-partial slots of an attention launch: unit + chunk, chunks <=
+// kMaxAttendChunks.
+inline size_t partial_slots(size_t units) { return units + kMaxAttendChunks; }
 
 cudaError_t launch_kv_append(const KvAppendParams& p, int head_dim, cudaStream_t stream);
 cudaError_t launch_build_meta(const BuildMetaParams& p, int head_dim, int num_sms,
                               cudaStream_t stream);
 cudaError_t launch_score(const ScoreParams& p, int head_dim, int num_sms, cudaStream_t stream);
-// The selection; with pm, extra CTAs also merge each unit's forced-list
-// partials (they run beside the selection CTAs).
-cudaError_t launch_select(const SelectParams& p, cudaStream_t stream,
-                          const PremergeParams* pm = nullptr);
-// sparse_decode's path: four kernels chained by programmatic dependent
-// launch (score + forced attention, select, selected attention, merge).
-cudaError_t launch_sparse_fused(const FusedParams& p, int head_dim, int num_sms,
-                                cudaStream_t stream, int stage = 0);
+cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
 // Attention over the list of each unit (dense: all pages; sparse: prefix,
-// selected, window), then the merge of the per-warp partials into out.
+// window, selected), then the merge of the split partials into out.  what:
+// kAttendAndMerge, or one of the two kernels alone (for stage timing).
+enum : int { kAttendAndMerge = 0, kAttendOnly = 1, kMergeOnly = 2 };
 cudaError_t launch_attend(AttendParams p, int head_dim, int num_sms, cudaStream_t stream,
-                          int* kernels_launched);
-// The attention alone: partials in slots p.slot_base + unit + chunk; sets
-// p.num_chunks (at most kMaxAttendChunks).
-cudaError_t launch_attend_partials(AttendParams& p, int head_dim, int num_sms,
-                                   cudaStream_t stream);
-// The chunk count launch_attend_partials uses.
-int attend_chunks(int head_dim, int num_sms);
+                          int what = kAttendAndMerge);
 
 }  // namespace slc

@@ -1,5 +1,5 @@
-// Candidate-page scoring building blocks shared by the scoring kernel
-// (slc_score.cu) and the fused sparse decode (slc_fused.cu): the Quest
+// Candidate-page scoring building blocks of the scoring kernel
+// (slc_score.cu): the Quest
 // upper bound of q.k over a page, summed over the query heads that share
 // the kv head ("Hybrid LLM Decoding 2.2x Faster at 256k, No Retraining",
 // section "The method: sliding window + prefix + query-aware pages,
