@@ -40,6 +40,39 @@ namespace {
 
 using namespace attn;
 
+// L2 prefetch of the K and V tiles of the prefix and window pages among
+// list positions [s, e) (sparse lists; every thread of the CTA calls it).
+template <int D>
+__device__ void prefetch_forced(const AttendParams& p, long long s, long long e) {
+    constexpr uint32_t TILE = kPage * D * 2;
+    if (s >= e) return;
+    auto len_of = [&](int b) { return list_len(p, b); };
+    int u;
+    long long ustart;
+    locate_unit(s, p.batch, p.hkv, len_of, &u, &ustart);  // warp-wide: every warp does it
+    while (s < e && u < p.batch * p.hkv) {
+        const int b = u / p.hkv, h = u % p.hkv;
+        const int len = list_len(p, b);
+        const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
+        const PageRanges r = page_ranges(L, p.prefix, p.window);
+        const int nforced = r.np + (r.n - r.ws);
+        const int i0 = (int)(s - ustart);
+        const int i1 = (int)(min(e, ustart + len) - ustart);
+        for (int i = i0 + (int)threadIdx.x; i < min(i1, nforced); i += blockDim.x) {
+            const int j = i < r.np ? i : r.ws + (i - r.np);
+            const int ph = p.block_table[(long long)b * p.max_pages + j];
+            if (ph >= 0 && ph < p.num_pages) {
+                const long long off = ((long long)ph * p.hkv + h) * TILE;
+                prefetch_l2(static_cast<const uint8_t*>(p.k_cache) + off, TILE);
+                prefetch_l2(static_cast<const uint8_t*>(p.v_cache) + off, TILE);
+            }
+        }
+        s = ustart + len;
+        ustart = s;
+        ++u;
+    }
+}
+
 // One CTA per chunk of the concatenated page lists.  For every unit piece
 // of the chunk, the CTA's warps take its pages round-robin, then combine
 // their partials in shared memory (reusing their rings) into one partial,
@@ -60,15 +93,19 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttendParams p) {
     }
     __syncwarp();
     grid_dep_launch();  // the merge may start; it waits before reading partials
-    // after a selection kernel, stream nothing before it is done: its
-    // latency-bound work runs without competing traffic
-    if (p.wait_first) grid_dep_wait();
 
     auto len_of = [&](int b) { return list_len(p, b); };
     const long long total = total_units(p.batch, p.hkv, len_of);
     const long long cpp = (total + gridDim.x - 1) / gridDim.x;
     const long long s = (long long)blockIdx.x * cpp;
     const long long e = min(total, s + cpp);
+    if (p.wait_first) {
+        // After a selection kernel: while it runs, only bring this chunk's
+        // prefix and window pages (known without the selection) into L2,
+        // then wait for the selection before any other read.
+        prefetch_forced<D>(p, s, e);
+        grid_dep_wait();
+    }
     uint32_t it = 0;
     bool ok = true;
     attend_range<D, NW, STAGES>(p, smem, ring, it, ok, s, e, blockIdx.x, 0, [](int) {});
