@@ -231,6 +231,88 @@ class Workload:
                                   dtype=torch.float32, device="cuda")
 
 
+def single_layer_entry(W, reps, flush, peak):
+    """Sparse and dense decode of one single-layer workload (eager calls,
+    L2 flushed before each)."""
+    import sparse_long_context_max_b200 as slc
+    x, wl = W.x, W.wl
+    lens = x.seq_lens.tolist()
+    sp = timed(lambda: slc.sparse_decode(W.q, W.cache, W.bt, W.sl, x.prefix, x.window, x.budget,
+                                         out=W.out, workspace=W.ws), reps, flush)
+    dn = timed(lambda: slc.dense_decode(W.q, W.cache, W.bt, W.sl, out=W.out, workspace=W.ws),
+               max(5, reps // 4), flush)
+    tb = algorithmic_bytes(lens, wl.hq, wl.hkv, wl.head_dim, x.prefix, x.window, x.budget)[0]
+    db = algorithmic_bytes(lens, wl.hq, wl.hkv, wl.head_dim, 0, 0, 0, True)[0]
+    gbs = tb / (sp * 1e-3) / 1e9
+    ctx = ("ctx %d" % wl.context if wl.context else
+           "ctx log-uniform in [%d, %d] (mean %d)" % (wl.ragged_lo, wl.ragged_hi,
+                                                      sum(lens) // len(lens)))
+    desc = ("B=%d, %s, Hq %d / Hkv %d, d %d, page 16, prefix %d, window %d, budget %d pages, "
+            "%s page pool" % (wl.batch, ctx, wl.hq, wl.hkv, wl.head_dim, x.prefix, x.window,
+                              x.budget, wl.layout))
+    return {"workload": desc, "sparse_us": round(sp * 1e3, 2), "dense_us": round(dn * 1e3, 2),
+            "speedup_vs_dense": round(dn / sp, 2), "algorithmic_bytes": tb,
+            "hbm_gbs": round(gbs, 1), "step_roofline_frac": round(gbs / peak, 4),
+            "dense_gbs": round(db / (dn * 1e-3) / 1e9, 1)}
+
+
+def layers_entry(reps, flush, peak):
+    """The 15-layer workload at 131072 tokens: every layer's decode
+    attention with its own (window, budget) -- or dense -- and its own
+    query, each timed alone with L2 flushed before it, then summed.  The
+    layers share one layer's cache: the time depends on the lengths, the
+    window and the budget, not on the values, and the flush removes any
+    reuse between layers.  For every sparse layer, reused_selection_us is
+    the same layer attending a selection it is given (slc_sparse_attend:
+    scoring and selection skipped), as a layer that reuses another layer's
+    indices would."""
+    import torch
+    import sparse_long_context_max_b200 as slc
+    import synth
+    W = Workload("layers131k")
+    wl, x = W.wl, W.x
+    B, hq, hkv, D = wl.batch, wl.hq, wl.hkv, wl.head_dim
+    lens = x.seq_lens.tolist()
+    plan = synth.layer_plan(wl)
+    kmax = max(k for _, k, _ in plan)
+    ws = torch.empty(slc.workspace_size(B, hq, hkv, D, x.block_table.shape[1], kmax),
+                     dtype=torch.uint8, device="cuda")
+    layers, total, dense_us = [], 0.0, None
+    for i, (window, budget, dense) in enumerate(plan):
+        q = synth.layer_query(wl, i).cuda()
+        if dense:
+            fn = lambda q=q: slc.dense_decode(q, W.cache, W.bt, W.sl, out=W.out, workspace=ws)
+            b = algorithmic_bytes(lens, hq, hkv, D, 0, 0, 0, True)[0]
+            t = timed(fn, max(5, reps // 4), flush)
+            dense_us = t * 1e3
+        else:
+            fn = lambda q=q, w=window, k=budget: slc.sparse_decode(
+                q, W.cache, W.bt, W.sl, wl.prefix, w, k, out=W.out, workspace=ws)
+            b = algorithmic_bytes(lens, hq, hkv, D, wl.prefix, window, budget)[0]
+            t = timed(fn, reps, flush)
+            # the same layer reusing a selection (score and select skipped)
+            sel = torch.empty((B, hkv, budget), dtype=torch.int32, device="cuda")
+            slc.sparse_decode(q, W.cache, W.bt, W.sl, wl.prefix, window, budget, out=W.out,
+                              selected_out=sel, workspace=ws)
+            shared = timed(lambda q=q, w=window, sel=sel: slc.sparse_attend(
+                q, W.cache, W.bt, W.sl, wl.prefix, w, sel, out=W.out, workspace=ws), reps, flush)
+        total += t * 1e3
+        e = {"layer": i, "window": window, "budget": budget, "dense": dense,
+             "us": round(t * 1e3, 2), "bytes": b, "gbs": round(b / (t * 1e-3) / 1e9, 1),
+             "frac": round(b / (t * 1e-3) / 1e9 / peak, 4)}
+        if not dense:
+            e["reused_selection_us"] = round(shared * 1e3, 2)
+        layers.append(e)
+    assert slc.device_status() == 0
+    entry = {"workload": "15 layers, B=4, ctx 131072, Hq 16 / Hkv 2, d 256, page 16, prefix 128, "
+                         "seeded (window, budget) per layer, 2 dense layers",
+             "attention_us_per_step": round(total, 2), "layers": layers}
+    if dense_us:
+        entry["all_dense_us_per_step"] = round(dense_us * len(plan), 2)
+        entry["speedup_vs_all_dense"] = round(dense_us * len(plan) / total, 2)
+    return entry
+
+
 def timed(fn, reps, flush, warm=3):
     """Average device time (ms) of fn() over reps, L2 flushed before each."""
     import torch
@@ -465,6 +547,15 @@ def run_ours(args, rank, world, local):
             "dense_gbs": round(db256 / (dn * 1e-3) / 1e9, 1),
             "stages": {STAGES[k]: stage_entry(k) for k in STAGES}}
         assert slc.device_status() == 0
+        del W256
+
+        # ---- the other workloads: tiny, ragged batch, 15-layer plan
+        for name in ("tiny", "ragged"):
+            Wx = Workload(name)
+            also[name] = dict(single_layer_entry(Wx, reps, flush, peak))
+            assert slc.device_status() == 0
+            del Wx
+        also["layers131k"] = layers_entry(reps, flush, peak)
 
     result = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,

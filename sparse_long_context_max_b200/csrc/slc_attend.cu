@@ -99,13 +99,12 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttendParams p) {
     const long long cpp = (total + gridDim.x - 1) / gridDim.x;
     const long long s = (long long)blockIdx.x * cpp;
     const long long e = min(total, s + cpp);
-    if (p.wait_first) {
-        // After a selection kernel: while it runs, only bring this chunk's
-        // prefix and window pages (known without the selection) into L2,
-        // then wait for the selection before any other read.
-        prefetch_forced<D>(p, s, e);
-        grid_dep_wait();
-    }
+    // After a selection kernel: while it runs, only bring this chunk's
+    // prefix and window pages (known without the selection) into L2.  Every
+    // read of data waits for the preceding kernel (which may be writing the
+    // selection, the cache, or reading the partial slots).
+    if (p.wait_first) prefetch_forced<D>(p, s, e);
+    grid_dep_wait();
     uint32_t it = 0;
     bool ok = true;
     attend_range<D, NW, STAGES>(p, smem, ring, it, ok, s, e, blockIdx.x, 0, [](int) {});

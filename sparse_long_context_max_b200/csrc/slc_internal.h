@@ -98,7 +98,7 @@ struct AttendParams {
     int prefix, window, budget;
     float scale_log2;  // softmax scale * log2(e)
     int num_chunks;    // chunks of the attention launch (one per CTA)
-    int wait_first;    // wait for the preceding kernel before any read (it wrote the selection)
+    int wait_first;    // the preceding kernel writes the selection: L2-prefetch the forced pages first
 };
 
 // Workspace carve-up shared by the API and the size query.

@@ -38,6 +38,7 @@ __all__ = [
     "Inputs",
     "make_inputs",
     "step_tokens",
+    "layer_query",
     "layer_plan",
     "chunk_seed",
 ]
@@ -220,7 +221,7 @@ def make_inputs(wl: Workload, layer: int = 0, fill: str = "zero",
     _fill_(kc, fill)
     _fill_(vc, fill)
 
-    q = _randn((B, Hq, D), seed, "q", 0).to(torch.bfloat16)
+    q = layer_query(wl, layer)
 
     CH = 256  # logical pages per generator chunk
     jobs = []
@@ -283,6 +284,12 @@ def make_inputs(wl: Workload, layer: int = 0, fill: str = "zero",
                   seq_lens=torch.tensor(lens, dtype=torch.int32),
                   needle_tokens=needle_tokens, prefix=wl.prefix, window=window,
                   budget=budget, layer=layer)
+
+
+def layer_query(wl: Workload, layer: int = 0) -> torch.Tensor:
+    """The decode query of ``layer`` (bf16 [B][Hq][D]), as make_inputs draws it."""
+    seed = wl.seed + 7919 * layer
+    return _randn((wl.batch, wl.hq, wl.head_dim), seed, "q", 0).to(torch.bfloat16)
 
 
 def step_tokens(wl: Workload, step: int, layer: int = 0):

@@ -137,6 +137,28 @@ def test_tiny_sparse_parity(tiny):
     check_output(x, out, x.prefix, x.window, sel)
 
 
+def test_sparse_attend_with_another_layers_selection():
+    """Cross-layer reuse of a selection ("IndexCache: cross-layer reuse speeds
+    30B prefill 1.82x": a Shared layer takes the indices of the preceding
+    Full layer): slc_sparse_attend, given a selection and another query,
+    attends the prefix, the window and exactly the given pages."""
+    import copy
+    import sparse_long_context_max_b200 as slc
+    # the short sequence has fewer candidates than the budget: -1 padding
+    x = small(3, 16, 4, 128, [5000, 2100, 900], prefix=64, window=256, budget=40, seed=21)
+    d = Dev(x)
+    _, sel = d.sparse()  # the Full layer's selection
+    q2 = torch.randn(x.q.shape, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    out = slc.sparse_attend(q2.cuda(), d.cache, d.bt, d.sl, x.prefix, x.window,
+                            torch.from_numpy(sel).cuda())
+    torch.cuda.synchronize()
+    assert slc.device_status() == 0
+    assert (sel[2] == -1).any()
+    y = copy.copy(x)
+    y.q = q2
+    check_output(y, out.cpu().double().numpy(), x.prefix, x.window, sel)
+
+
 def test_stages_in_order_equal_one_call():
     """slc_sparse_decode_stage 1..4 on one workspace reproduce slc_sparse_decode
     bit for bit (same kernels, same order)."""
