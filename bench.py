@@ -644,7 +644,7 @@ def run_reference(args, rank, world):
 def run_profile(name):
     """Each entry point twice on one workload, nothing timed: the command
     that ncu captures.  Launch order: build_meta, then twice (kv_append,
-    score_forced, select, attend, merge), then dense (attend, merge)."""
+    score, select, attend, merge), then dense (attend, merge)."""
     import torch
     import sparse_long_context_max_b200 as slc
     w = Workload(name, extra_tokens=2)
