@@ -283,6 +283,28 @@ def test_layout_invariance():
         np.testing.assert_array_equal(u, w)
 
 
+def test_units_are_independent():
+    # one (sequence, kv head) unit alone -- its pages, its query group, one
+    # kv head -- gives that unit's slice of the whole step (the selection is
+    # per unit), which is what the threaded CPU baseline relies on
+    x = _small_cache(3, 8, 2, 32, [300, 190, 77], layout="shuffled", seed=16)
+    P, W, K = 16, 48, 3
+    G = 4
+    out, sel, nsel = oracle.sparse_decode(x.q, x.k_cache, x.v_cache, x.block_table,
+                                          x.seq_lens, P, W, K)
+    for b, L in enumerate(x.seq_lens.tolist()):
+        n = -(-L // 16)
+        phys = x.block_table[b, :n].long()
+        for h in range(2):
+            o, s_, ns = oracle.sparse_decode(
+                x.q[b:b + 1, h * G:(h + 1) * G].contiguous(),
+                x.k_cache[phys, h:h + 1].contiguous(), x.v_cache[phys, h:h + 1].contiguous(),
+                torch.arange(n, dtype=torch.int32).reshape(1, n), x.seq_lens[b:b + 1], P, W, K)
+            np.testing.assert_array_equal(o[0], out[b, h * G:(h + 1) * G])
+            np.testing.assert_array_equal(s_[0, 0], sel[b, h])
+            assert ns[0, 0] == nsel[b, h]
+
+
 def test_composition_of_steps():
     x = _small_cache(2, 4, 2, 32, [300, 190], seed=15)
     P, W, K = 32, 40, 3
