@@ -262,14 +262,16 @@ def layers_entry(reps, flush, peak):
     query, each timed alone with L2 flushed before it, then summed.  The
     layers share one layer's cache: the time depends on the lengths, the
     window and the budget, not on the values, and the flush removes any
-    reuse between layers.  For every sparse layer, reused_selection_us is
+    reuse between layers.  graph_us_per_step then times a whole decode step
+    of the plan -- every layer's append and decode, each layer on its own
+    cache -- captured as one CUDA graph.  For every sparse layer, reused_selection_us is
     the same layer attending a selection it is given (slc_sparse_attend:
     scoring and selection skipped), as a layer that reuses another layer's
     indices would."""
     import torch
     import sparse_long_context_max_b200 as slc
     import synth
-    W = Workload("layers131k")
+    W = Workload("layers131k", extra_tokens=16)  # room for one appended token
     wl, x = W.wl, W.x
     B, hq, hkv, D = wl.batch, wl.hq, wl.hkv, wl.head_dim
     lens = x.seq_lens.tolist()
@@ -304,9 +306,45 @@ def layers_entry(reps, flush, peak):
             e["reused_selection_us"] = round(shared * 1e3, 2)
         layers.append(e)
     assert slc.device_status() == 0
+
+    # one decode step of the whole plan as one CUDA graph: per layer, the new
+    # token's append to that layer's own cache (a device copy of the drawn
+    # one, so no layer finds another's data in L2), then that layer's decode
+    caches = []
+    for _ in plan:
+        c = slc.PagedCache(W.k.clone(), W.v.clone())
+        slc.build_page_meta(c, W.bt, W.sl)
+        caches.append(c)
+    pos = W.sl.clone()  # the same slot every replay: the append is idempotent
+    lens1 = (W.sl + 1).contiguous()
+    toks = [synth.step_tokens(wl, 1, layer=i) for i in range(len(plan))]
+    qs = [t[0].cuda() for t in toks]
+    kns = [t[1].cuda() for t in toks]
+    vns = [t[2].cuda() for t in toks]
+    outs = [torch.empty_like(W.out) for _ in plan]
+
+    def step():
+        for i, (window, budget, dense) in enumerate(plan):
+            slc.kv_append(caches[i], kns[i], vns[i], W.bt, pos)
+            if dense:
+                slc.dense_decode(qs[i], caches[i], W.bt, lens1, out=outs[i], workspace=ws)
+            else:
+                slc.sparse_decode(qs[i], caches[i], W.bt, lens1, wl.prefix, window, budget,
+                                  out=outs[i], workspace=ws)
+
+    g = graph_of(step)
+    t_graph = timed(g.replay, max(5, reps // 2), flush)
+    assert slc.device_status() == 0
+    launches = sum(1 + (2 if dense else slc.KERNELS_PER_CALL["sparse_decode"])
+                   for _, _, dense in plan)
+    del g, caches
     entry = {"workload": "15 layers, B=4, ctx 131072, Hq 16 / Hkv 2, d 256, page 16, prefix 128, "
                          "seeded (window, budget) per layer, 2 dense layers",
-             "attention_us_per_step": round(total, 2), "layers": layers}
+             "attention_us_per_step": round(total, 2),
+             "graph_us_per_step": round(t_graph * 1e3, 2),
+             "graph_step": "one CUDA graph: per layer kv_append + decode, each layer on its own "
+                           "cache; %d kernel launches" % launches,
+             "layers": layers}
     if dense_us:
         entry["all_dense_us_per_step"] = round(dense_us * len(plan), 2)
         entry["speedup_vs_all_dense"] = round(dense_us * len(plan) / total, 2)
