@@ -77,8 +77,10 @@ __device__ void prefetch_forced(const AttendParams& p, long long s, long long e)
 // of the chunk, the CTA's warps take its pages round-robin, then combine
 // their partials in shared memory (reusing their rings) into one partial,
 // stored in slot (unit + chunk).
+// Residency: three CTAs per SM at d = 128 (64 KB of rings each), one at
+// d = 256; the register budget follows.
 template <int D, int NW, int STAGES>
-__global__ void __launch_bounds__(NW * 32) attend_kernel(AttendParams p) {
+__global__ void __launch_bounds__(NW * 32, D == 128 ? 3 : 1) attend_kernel(AttendParams p) {
     constexpr int TILE = kPage * D * 2;
     constexpr int RING = STAGES * 2 * TILE;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -107,7 +109,7 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttendParams p) {
     grid_dep_wait();
     uint32_t it = 0;
     bool ok = true;
-    attend_range<D, NW, STAGES>(p, smem, ring, it, ok, s, e, blockIdx.x, 0, [](int) {});
+    attend_range<D, NW, STAGES>(p, smem, ring, it, ok, s, e, blockIdx.x);
 }
 
 // Merge of the CTA partials of one (unit, query head): slots unit + chunk

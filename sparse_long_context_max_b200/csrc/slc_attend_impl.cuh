@@ -20,29 +20,18 @@ struct Ring {
 };
 
 // A unit's list (AttendParams::list):
-//   kListDense     pages 0..n-1;
-//   kListSparse    prefix pages, window pages, then the selected pages
-//                  (forced pages first, so they need no selection);
-//   kListForced    prefix pages, then window pages;
-//   kListSelected  the selected pages alone.
-__device__ __forceinline__ bool list_is_selected(const AttendParams& p, const PageRanges& r,
-                                                 int i) {
-    if (p.list == kListSelected) return true;
-    return p.list == kListSparse && i >= r.np + (r.n - r.ws);
-}
+//   kListDense   pages 0..n-1;
+//   kListSparse  prefix pages, window pages, then the selected pages.
 
 // Logical page of list position i of a unit (and whether it is sane).
 __device__ __forceinline__ int list_page(const AttendParams& p, int u, const PageRanges& r,
                                          int i, bool* ok) {
     *ok = true;
     if (p.list == kListDense) return i;
-    int k = i;  // position within the selection
-    if (p.list != kListSelected) {
-        if (i < r.np) return i;
-        const int nwin = r.n - r.ws;
-        if (p.list == kListForced || i < r.np + nwin) return r.ws + (i - r.np);
-        k = i - r.np - nwin;
-    }
+    if (i < r.np) return i;
+    const int nwin = r.n - r.ws;
+    if (i < r.np + nwin) return r.ws + (i - r.np);
+    const int k = i - r.np - nwin;  // position within the selection
     const int j = __ldcg(p.selected + (long long)u * p.budget + k);
     if (j < r.np || j >= r.ws) {
         *ok = false;
@@ -119,14 +108,10 @@ __device__ void warp_attend(const AttendParams& p, const Ring& ring, uint32_t& i
     const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
     const PageRanges r = page_ranges(L, p.prefix, p.window);
 
-    // page ids of this warp's pages, 32 at a time: lane t holds page k0 + t.
-    // Selected pages come from the preceding (selection) kernel: wait for
-    // it only when a batch holds one.
+    // page ids of this warp's pages, 32 at a time: lane t holds page k0 + t
     int id_phys = 0, id_nv = 0;
     auto load_ids = [&](int k0) {
         const int k = k0 + lane;
-        const bool sel = k < npg && list_is_selected(p, r, i0 + k * stride);
-        if (__any_sync(0xffffffffu, sel)) grid_dep_wait();
         if (k < npg) resolve_page(p, u, b, r, L, i0 + k * stride, &id_phys, &id_nv);
     };
     load_ids(0);
@@ -279,13 +264,8 @@ __device__ void warp_attend(const AttendParams& p, const Ring& ring, uint32_t& i
 __device__ __forceinline__ int list_len(const AttendParams& p, int b) {
     const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
     const PageRanges r = page_ranges(L, p.prefix, p.window);
-    const int forced = r.np + (r.n - r.ws), sel = min(p.budget, r.ws - r.np);
-    switch (p.list) {
-        case kListDense: return r.n;
-        case kListForced: return forced;
-        case kListSelected: return sel;
-        default: return forced + sel;
-    }
+    if (p.list == kListDense) return r.n;
+    return r.np + (r.n - r.ws) + min(p.budget, r.ws - r.np);
 }
 
 // Combine the NW warp partials of one unit piece (each warp's WarpState,
@@ -348,13 +328,13 @@ __device__ __forceinline__ void cta_store_partial(const AttendParams& p, uint8_t
 
 // Attend positions [s, e) of the concatenated lists of all units with the
 // CTA's NW warps (each warp: ring of STAGES stages at smem + warp * RING).
-// before(unit) is called by every thread before a unit piece; every piece
-// yields one partial, stored in slot slot_base + unit + chunk.
-template <int D, int NW, int STAGES, class Before>
+// Every unit piece yields one partial, stored in slot unit + chunk.  The
+// caller has waited for the preceding kernel (which may write the
+// selection or the cache, or read the partial slots).
+template <int D, int NW, int STAGES>
 __device__ __forceinline__ void attend_range(const AttendParams& p, uint8_t* smem,
                                              const Ring& ring, uint32_t& it, bool& ok,
-                                             long long s, long long e, long long chunk,
-                                             long long slot_base, Before before) {
+                                             long long s, long long e, long long chunk) {
     constexpr int RING = STAGES * 2 * kPage * D * 2;
     const int warp = threadIdx.x >> 5;
     if (s >= e) return;
@@ -371,10 +351,8 @@ __device__ __forceinline__ void attend_range(const AttendParams& p, uint8_t* sme
         }
         const int i0 = (int)(s - ustart);
         const int i1 = (int)(min(e, ustart + len) - ustart);
-        before(u);
         warp_attend<D, STAGES>(p, ring, it, ok, u, i0 + warp, i1, NW, st);
-        grid_dep_wait();  // partial slots may still be read by a preceding merge
-        cta_store_partial<D, NW, RING>(p, smem, st, slot_base + u + chunk);
+        cta_store_partial<D, NW, RING>(p, smem, st, u + chunk);
         s = ustart + len;
         ustart = s;
         ++u;

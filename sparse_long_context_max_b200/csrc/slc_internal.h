@@ -80,7 +80,7 @@ constexpr int kSelTile = 16;
 inline int cand_stride_of(int max_pages) { return (max_pages + 63) / 64 * 64; }
 
 // Page list attended per unit (see slc_attend_impl.cuh).
-enum : int { kListDense = 0, kListSparse = 1, kListForced = 2, kListSelected = 3 };
+enum : int { kListDense = 0, kListSparse = 1 };
 
 struct AttendParams {
     const void* q;
@@ -94,7 +94,7 @@ struct AttendParams {
     float* out;               // [B][Hq][D]
     unsigned* status;
     int batch, hq, hkv, group, max_pages, num_pages;
-    int list;  // kListDense, kListSparse, kListForced or kListSelected
+    int list;  // kListDense or kListSparse
     int prefix, window, budget;
     float scale_log2;  // softmax scale * log2(e)
     int num_chunks;    // chunks of the attention launch (one per CTA)
