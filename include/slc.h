@@ -50,6 +50,11 @@
  * positions) are range-checked by the kernels: a bad entry is skipped and
  * flagged in the device status word instead of being dereferenced.
  *
+ * Devices.  A process drives one GPU: each kernel's shared-memory limit and
+ * occupancy are set and looked up once, on the first call, for the device
+ * current then (one process per GPU, as under torchrun).  A call made later
+ * with another device current may fail with SLC_ERR_CUDA.
+ *
  * Errors.  0 on success; a negative SLC_ERR_* code otherwise.
  */
 #ifndef SLC_H
