@@ -173,9 +173,13 @@ SLC_API int slc_sparse_decode_stage(int32_t stage, const void *q, const slc_cach
 
 /* Attention over the prefix pages, the window pages and a caller-given
  * selection (same layout as slc_select_pages writes: [batch][num_kv_heads]
- * [budget] ascending logical pages, -1 padded; entries must be candidate
- * pages), then the merge of the split partials.  This is the back half of
- * slc_sparse_decode; it also lets a layer reuse another layer's selection. */
+ * [budget] ascending logical pages, -1 padded), then the merge of the split
+ * partials.  The first min(budget, #candidates) entries of each row are
+ * read, and each must be a candidate page of this call's prefix and window;
+ * an entry that is not is skipped and flagged (SLC_STATUS_BAD_SELECTION in
+ * the status word).  This is the back half of slc_sparse_decode; it also
+ * lets a layer reuse the selection of another layer with the same lengths,
+ * prefix and window. */
 SLC_API int slc_sparse_attend(const void *q, const slc_cache_t *cache, const int32_t *block_table,
                       int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
                       int32_t num_q_heads, int32_t prefix, int32_t window, int32_t budget,
