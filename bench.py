@@ -543,8 +543,10 @@ def run_ours(args, rank, world, local):
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(outh.numel() * 4),
            "path": "binding calls kv_append + sparse_decode (eager), pinned host copies"}
 
-    # ---- 256k workload: sparse vs dense, per-kernel roofline
-    if not args.no_also:
+    # ---- 256k workload: sparse vs dense, per-kernel roofline (one GPU only:
+    # under torchrun every rank would hold its GPU through these extra
+    # single-GPU measurements, which the scaling line does not use)
+    if not args.no_also and world == 1:
         del qs, kns, vns
         W256 = Workload("decode256k")
         y = W256.x
