@@ -31,8 +31,8 @@ __all__ = [
 
 PAGE = 16
 
-# kernels one call launches (sparse: score with forced attention, select, attend,
-# merge; dense and attend: attend, merge)
+# kernels one call launches (sparse: score, select, attend, merge; dense and
+# attend: attend, merge)
 KERNELS_PER_CALL = {"sparse_decode": 4, "sparse_decode_stage": 1, "dense_decode": 2,
                     "sparse_attend": 2, "kv_append": 1,
                     "build_page_meta": 1, "score_pages": 1, "select_pages": 1}
