@@ -97,21 +97,24 @@ def algorithmic_bytes(lens, hq, hkv, D, prefix, window, budget, dense=False):
 
 
 def stage_bytes(lens, hq, hkv, D, prefix, window, budget):
-    """Algorithmic bytes of the two HBM-bound stages of sparse_decode:
-    stage 1 reads the candidates' metadata and q; stage 3 reads the K and V
-    of the prefix, window and selected pages and q."""
-    meta = kv = 0
+    """Algorithmic bytes of the two kernels of sparse_decode: stage 1 (the
+    streaming kernel) reads the candidates' metadata, the K and V of the
+    prefix and window pages, and q; stage 2 (the finishing kernel) reads the
+    K and V of the selected pages and q, and writes out."""
+    meta = forced = sel = 0
     for L in lens:
         n, np_, ws = page_ranges(L, prefix, window)
         nc = ws - np_
         meta += nc * hkv * 4 * D
-        kv += (min(L, 16 * np_) + max(0, L - 16 * ws) + 16 * min(budget, nc)) * hkv * 4 * D
+        forced += (min(L, 16 * np_) + max(0, L - 16 * ws)) * hkv * 4 * D
+        sel += 16 * min(budget, nc) * hkv * 4 * D
     qb = len(lens) * hq * D * 2
-    return {1: meta + qb, 3: kv + qb}
+    ob = len(lens) * hq * D * 4
+    return {1: meta + forced + qb, 2: sel + qb + ob}
 
 
-STAGES = {1: "score", 2: "select", 3: "attend", 4: "merge"}
-STAGE_KERNELS = {1: "score_kernel", 2: "select_kernel", 3: "attend_kernel", 4: "merge_kernel"}
+STAGES = {1: "stream", 2: "finish"}
+STAGE_KERNELS = {1: "stream_kernel", 2: "finish_kernel"}
 
 
 class Clocks:
@@ -486,7 +489,7 @@ def run_ours(args, rank, world, local):
 
     kt = stage_times(W64, cur_q, cur_len, x)
     kb = stage_bytes(lens64, hq, hkv, D, x.prefix, x.window, x.budget)
-    dom = max((1, 3), key=lambda k: kt[k])  # the slower HBM-bound stage
+    dom = max((1, 2), key=lambda k: kt[k])  # the slower stage
     ach = kb[dom] / (kt[dom] * 1e-3) / 1e9
     roofline = {"kernel": STAGE_KERNELS[dom], "stage": STAGES[dom], "bound": "hbm",
                 "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",

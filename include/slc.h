@@ -50,10 +50,10 @@
  * positions) are range-checked by the kernels: a bad entry is skipped and
  * flagged in the device status word instead of being dereferenced.
  *
- * Devices.  A process drives one GPU: each kernel's shared-memory limit and
- * occupancy are set and looked up once, on the first call, for the device
- * current then (one process per GPU, as under torchrun).  A call made later
- * with another device current may fail with SLC_ERR_CUDA.
+ * Devices.  Calls run on the device current on the calling thread.  Each
+ * kernel's shared-memory limit, occupancy and cluster capacity are looked
+ * up once per device, on the first call made with that device current
+ * (make that first call before any stream capture).
  *
  * Errors.  0 on success; a negative SLC_ERR_* code otherwise.
  */
@@ -145,24 +145,30 @@ SLC_API int slc_select_pages(const float *scores, int32_t num_kv_heads, int32_t 
                      const int32_t *seq_lens, int32_t batch, int32_t prefix, int32_t window,
                      int32_t budget, int32_t *selected, slc_stream_t stream);
 
-/* One decode step of one layer: score -> select -> attend prefix, window
- * and selected pages -> merge the split partials.  scale <= 0 means
- * 1/sqrt(head_dim).  selected_out (nullable) receives the selection as
- * slc_select_pages writes it.  workspace: device, >= slc_workspace_size(). */
+/* One decode step of one layer, in two kernels:
+ *   1 (streaming)  attention over the prefix and window pages, and the
+ *                  scores of the candidate pages (all SMs, HBM-bound);
+ *   2 (finishing)  per unit, on one thread-block cluster: the selection,
+ *                  attention over the selected pages, and the merge of all
+ *                  partials into out.
+ * scale <= 0 means 1/sqrt(head_dim).  selected_out (nullable) receives the
+ * selection as slc_select_pages writes it.  workspace: device, >=
+ * slc_workspace_size().  A nonzero device status word after the call
+ * (slc_device_status) means out and selected_out may be invalid. */
 SLC_API int slc_sparse_decode(const void *q, const slc_cache_t *cache, const int32_t *block_table,
                       int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
                       int32_t num_q_heads, int32_t prefix, int32_t window, int32_t budget,
                       float scale, float *out, int32_t *selected_out, void *workspace,
                       size_t workspace_bytes, slc_stream_t stream);
 
-/* One stage of slc_sparse_decode alone (same arguments), for timing and
- * inspection; the stages run in this order and each reads what the earlier
- * ones left in the workspace (and in selected_out):
- *   1  score the candidate pages
- *   2  select the pages
- *   3  attend the prefix, window and selected pages
- *   4  merge the split partials into out
- * Running 1, 2, 3, 4 in order equals one slc_sparse_decode call.  Returns
+/* One of the two kernels of slc_sparse_decode alone (same arguments), for
+ * timing and inspection:
+ *   1  the streaming kernel: prefix/window attention partials and candidate
+ *      scores, left in the workspace;
+ *   2  the finishing kernel: selection (into selected_out when given),
+ *      selected-page attention and the merge into out, from what stage 1
+ *      left in the same workspace.
+ * Running 1 then 2 equals one slc_sparse_decode call.  Returns
  * SLC_ERR_INVALID_ARG for any other stage. */
 SLC_API int slc_sparse_decode_stage(int32_t stage, const void *q, const slc_cache_t *cache,
                             const int32_t *block_table, int32_t max_pages_per_seq,
@@ -173,13 +179,15 @@ SLC_API int slc_sparse_decode_stage(int32_t stage, const void *q, const slc_cach
 
 /* Attention over the prefix pages, the window pages and a caller-given
  * selection (same layout as slc_select_pages writes: [batch][num_kv_heads]
- * [budget] ascending logical pages, -1 padded), then the merge of the split
- * partials.  The first min(budget, #candidates) entries of each row are
- * read, and each must be a candidate page of this call's prefix and window;
- * an entry that is not is skipped and flagged (SLC_STATUS_BAD_SELECTION in
- * the status word).  This is the back half of slc_sparse_decode; it also
- * lets a layer reuse the selection of another layer with the same lengths,
- * prefix and window. */
+ * [budget] ascending logical pages, -1 padded).  The attended set is the
+ * union: every entry j with 0 <= j < n_b is attended once (an entry that is
+ * itself a prefix or window page of this call adds nothing), -1 entries are
+ * padding, and an entry that is out of range or not above the entry before
+ * it is skipped and flagged (SLC_STATUS_BAD_SELECTION).  This lets a layer
+ * reuse the selection of another layer of the same sequences -- cross-layer
+ * index reuse ("IndexCache: cross-layer reuse speeds 30B prefill 1.82x":
+ * Shared layers take the top-k of the nearest Full layer) -- even when the
+ * two layers' windows differ. */
 SLC_API int slc_sparse_attend(const void *q, const slc_cache_t *cache, const int32_t *block_table,
                       int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
                       int32_t num_q_heads, int32_t prefix, int32_t window, int32_t budget,

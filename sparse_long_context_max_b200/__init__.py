@@ -31,9 +31,9 @@ __all__ = [
 
 PAGE = 16
 
-# kernels one call launches (sparse: score, select, attend, merge; dense and
-# attend: attend, merge)
-KERNELS_PER_CALL = {"sparse_decode": 4, "sparse_decode_stage": 1, "dense_decode": 2,
+# kernels one call launches (sparse decode and sparse attend: the streaming
+# kernel, then the finishing kernel; dense: attend, merge)
+KERNELS_PER_CALL = {"sparse_decode": 2, "sparse_decode_stage": 1, "dense_decode": 2,
                     "sparse_attend": 2, "kv_append": 1,
                     "build_page_meta": 1, "score_pages": 1, "select_pages": 1}
 
@@ -228,9 +228,10 @@ def sparse_decode(q, cache: PagedCache, block_table, seq_lens, prefix, window, b
 
 def sparse_decode_stage(stage, q, cache: PagedCache, block_table, seq_lens, prefix, window,
                         budget, scale=0.0, out=None, selected_out=None, workspace=None):
-    """One stage (1 score + prefix/window attention, 2 select, 3 selected
-    attention, 4 merge) of sparse_decode alone; stages 1..4 in order equal
-    one sparse_decode call on the same workspace."""
+    """One of the two kernels of sparse_decode alone: stage 1 the streaming
+    kernel (prefix/window attention and candidate scores), stage 2 the
+    finishing kernel (selection, selected-page attention, merge).  Stages 1
+    then 2 on the same workspace equal one sparse_decode call."""
     _need(q, torch.bfloat16, "q", 3)
     _need(block_table, torch.int32, "block_table", 2)
     _need(seq_lens, torch.int32, "seq_lens", 1)
@@ -254,7 +255,8 @@ def sparse_decode_stage(stage, q, cache: PagedCache, block_table, seq_lens, pref
 def sparse_attend(q, cache: PagedCache, block_table, seq_lens, prefix, window, selected,
                   scale=0.0, out=None, workspace=None):
     """Attention over prefix, window and the given selection (int32
-    [B][Hkv][budget], ascending, -1 padded); returns out (fp32 [B][Hq][D])."""
+    [B][Hkv][budget], ascending, -1 padded; entries that are prefix or window
+    pages add nothing); returns out (fp32 [B][Hq][D])."""
     _need(q, torch.bfloat16, "q", 3)
     _need(block_table, torch.int32, "block_table", 2)
     _need(seq_lens, torch.int32, "seq_lens", 1)

@@ -19,13 +19,12 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
-struct DeviceInfo {
+struct DeviceSlot {
     bool ready;
-    int num_sms;
-    unsigned* status;
+    DeviceCfg cfg;
 };
 
-DeviceInfo g_devices[kMaxDevices];
+DeviceSlot g_devices[kMaxDevices];
 std::mutex g_mutex;
 thread_local char g_cuda_error[256];
 
@@ -35,23 +34,32 @@ int note_cuda(cudaError_t e, const char* where = "") {
     return SLC_ERR_CUDA;
 }
 
-// Per-device facts, looked up on the first call made with that device
-// current.
-int device_info(DeviceInfo** out) {
+// Per-device facts and launch settings (shared-memory limits, occupancies,
+// co-resident clusters), set up once per device on the first call made with
+// that device current.
+int device_cfg(const DeviceCfg** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return note_cuda(e);
     if (dev < 0 || dev >= kMaxDevices) return SLC_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_mutex);
-    DeviceInfo& d = g_devices[dev];
+    DeviceSlot& d = g_devices[dev];
     if (!d.ready) {
-        e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+        DeviceCfg c{};
+        c.device = dev;
+        e = cudaDeviceGetAttribute(&c.num_sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return note_cuda(e);
-        e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), slc_status_word);
+        e = cudaGetSymbolAddress(reinterpret_cast<void**>(&c.status), slc_status_word);
         if (e != cudaSuccess) return note_cuda(e);
+        if ((e = setup_score(c)) != cudaSuccess) return note_cuda(e, "setup score");
+        if ((e = setup_select(c)) != cudaSuccess) return note_cuda(e, "setup select");
+        if ((e = setup_attend(c)) != cudaSuccess) return note_cuda(e, "setup attend");
+        if ((e = setup_stream(c)) != cudaSuccess) return note_cuda(e, "setup stream");
+        if ((e = setup_finish(c)) != cudaSuccess) return note_cuda(e, "setup finish");
+        d.cfg = c;
         d.ready = true;
     }
-    *out = &d;
+    *out = &d.cfg;
     return SLC_OK;
 }
 
@@ -88,7 +96,11 @@ WorkspaceLayout workspace_layout(int batch, int hq, int hkv, int head_dim, int m
     size_t off = 0;
     w.scores = off;  // by candidate, in rows of cand_stride_of(max_pages)
     off = round_up(off + units * (size_t)cand_stride_of(max_pages) * sizeof(float), 256);
+    w.tile_max = off;  // one key per 16 candidates
+    off = round_up(off + units * (size_t)(cand_stride_of(max_pages) / kSelTile) * 4, 256);
     w.selected = off;
+    off = round_up(off + units * (size_t)(budget > 0 ? budget : 1) * sizeof(int32_t), 256);
+    w.sel_phys = off;
     off = round_up(off + units * (size_t)(budget > 0 ? budget : 1) * sizeof(int32_t), 256);
     w.part_acc = off;
     off = round_up(off + slots * group * head_dim * sizeof(float), 256);
@@ -138,8 +150,8 @@ int slc_kv_append(const slc_cache_t* cache, const void* k_new, const void* v_new
     if (batch == 0) return SLC_OK;
     if (!k_new || !v_new || !block_table || !positions) return SLC_ERR_INVALID_ARG;
     if (!aligned16(k_new) || !aligned16(v_new)) return SLC_ERR_INVALID_ARG;
-    DeviceInfo* dev;
-    if ((rc = device_info(&dev))) return rc;
+    const DeviceCfg* dev;
+    if ((rc = device_cfg(&dev))) return rc;
     KvAppendParams p{k_new,     v_new,     cache->k_cache,          cache->v_cache,
                      cache->meta, block_table, positions,            dev->status,
                      batch,     cache->num_kv_heads, max_pages_per_seq, cache->num_pages};
@@ -155,11 +167,11 @@ int slc_build_page_meta(const slc_cache_t* cache, const int32_t* block_table,
     if (batch < 0 || max_pages_per_seq <= 0) return SLC_ERR_INVALID_ARG;
     if (batch == 0) return SLC_OK;
     if (!block_table || !seq_lens) return SLC_ERR_INVALID_ARG;
-    DeviceInfo* dev;
-    if ((rc = device_info(&dev))) return rc;
+    const DeviceCfg* dev;
+    if ((rc = device_cfg(&dev))) return rc;
     BuildMetaParams p{cache->k_cache, cache->meta, block_table, seq_lens, dev->status, batch,
                       cache->num_kv_heads, max_pages_per_seq, cache->num_pages};
-    cudaError_t e = launch_build_meta(p, cache->head_dim, dev->num_sms, stream);
+    cudaError_t e = launch_build_meta(p, cache->head_dim, *dev, stream);
     return e == cudaSuccess ? SLC_OK : note_cuda(e);
 }
 
@@ -174,13 +186,13 @@ int slc_score_pages(const void* q, const slc_cache_t* cache, const int32_t* bloc
         return SLC_ERR_INVALID_ARG;
     if (batch == 0) return SLC_OK;
     if (!q || !block_table || !seq_lens || !scores || !aligned16(q)) return SLC_ERR_INVALID_ARG;
-    DeviceInfo* dev;
-    if ((rc = device_info(&dev))) return rc;
+    const DeviceCfg* dev;
+    if ((rc = device_cfg(&dev))) return rc;
     ScoreParams p{q,           cache->meta, block_table, seq_lens,
                   scores,      dev->status, batch,
                   num_q_heads, cache->num_kv_heads, num_q_heads / cache->num_kv_heads,
-                  max_pages_per_seq, cache->num_pages, prefix, window, 0};
-    cudaError_t e = launch_score(p, cache->head_dim, dev->num_sms, stream);
+                  max_pages_per_seq, cache->num_pages, prefix, window, 0, nullptr};
+    cudaError_t e = launch_score(p, cache->head_dim, *dev, stream);
     return e == cudaSuccess ? SLC_OK : note_cuda(e);
 }
 
@@ -193,17 +205,45 @@ int slc_select_pages(const float* scores, int32_t num_kv_heads, int32_t max_page
     if (max_pages_per_seq > kMaxCandidates) return SLC_ERR_UNSUPPORTED;
     if (batch == 0 || budget == 0) return SLC_OK;
     if (!scores || !seq_lens || !selected) return SLC_ERR_INVALID_ARG;
-    DeviceInfo* dev;
+    const DeviceCfg* dev;
     int rc;
-    if ((rc = device_info(&dev))) return rc;
+    if ((rc = device_cfg(&dev))) return rc;
     SelectParams p{scores, seq_lens, selected, dev->status, batch, num_kv_heads,
                    max_pages_per_seq, prefix, window, budget, 0};
     cudaError_t e = launch_select(p, stream);
     return e == cudaSuccess ? SLC_OK : note_cuda(e);
 }
 
-// mode: 0 dense, 1 sparse (score + select + attend), 2 sparse attend over
-// the caller's selection in `selected_out`.
+// mode: 0 dense, 1 sparse (stream: prefix/window attention + scores;
+// finish: select, attend the selection, merge), 2 sparse attention over the
+// caller's selection in `selected_out`.  stage (mode 1): 0 both kernels, 1
+// the streaming kernel alone, 2 the finishing kernel alone.
+// Argument checks of decode() apart from the workspace (which the caller
+// checks), in the order the codes are documented; nothing touches the GPU.
+// *nothing_to_do is set for an empty batch.
+static int check_decode(int mode, const void* q, const slc_cache_t* cache,
+                        const int32_t* block_table, int32_t max_pages_per_seq,
+                        const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                        int32_t prefix, int32_t window, int32_t budget, float scale,
+                        const float* out, const int32_t* selected_out, bool* nothing_to_do) {
+    *nothing_to_do = false;
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if ((rc = check_heads(cache, num_q_heads))) return rc;
+    if (batch < 0 || max_pages_per_seq <= 0 || prefix < 0 || window < 0 || budget < 0)
+        return SLC_ERR_INVALID_ARG;
+    if (mode != 0 && max_pages_per_seq > kMaxCandidates) return SLC_ERR_UNSUPPORTED;
+    if (!(scale == scale) || isinf(scale)) return SLC_ERR_INVALID_ARG;
+    if (batch == 0) {
+        *nothing_to_do = true;
+        return SLC_OK;
+    }
+    if (!q || !block_table || !seq_lens || !out) return SLC_ERR_INVALID_ARG;
+    if (mode == 2 && budget > 0 && !selected_out) return SLC_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out)) return SLC_ERR_INVALID_ARG;
+    return SLC_OK;
+}
+
 static int decode(int mode, const void* q, const slc_cache_t* cache,
                   const int32_t* block_table, int32_t max_pages_per_seq,
                   const int32_t* seq_lens, int32_t batch, int32_t num_q_heads, int32_t prefix,
@@ -211,34 +251,25 @@ static int decode(int mode, const void* q, const slc_cache_t* cache,
                   int32_t* selected_out, void* workspace, size_t workspace_bytes,
                   cudaStream_t stream, int stage = 0) {
     const bool sparse = mode != 0;
-    int rc = check_cache(cache);
-    if (rc) return rc;
-    if ((rc = check_heads(cache, num_q_heads))) return rc;
-    if (batch < 0 || max_pages_per_seq <= 0 || prefix < 0 || window < 0 || budget < 0)
-        return SLC_ERR_INVALID_ARG;
-    if (sparse && max_pages_per_seq > kMaxCandidates) return SLC_ERR_UNSUPPORTED;
-    if (!(scale == scale) || isinf(scale)) return SLC_ERR_INVALID_ARG;
-    if (batch == 0) return SLC_OK;
-    if (!q || !block_table || !seq_lens || !out || !workspace) return SLC_ERR_INVALID_ARG;
-    if (mode == 2 && budget > 0 && !selected_out) return SLC_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return SLC_ERR_INVALID_ARG;
+    bool empty;
+    int rc = check_decode(mode, q, cache, block_table, max_pages_per_seq, seq_lens, batch,
+                          num_q_heads, prefix, window, budget, scale, out, selected_out, &empty);
+    if (rc || empty) return rc;
+    if (!workspace || !aligned16(workspace)) return SLC_ERR_INVALID_ARG;
     const int hkv = cache->num_kv_heads, D = cache->head_dim;
     const WorkspaceLayout w =
         workspace_layout(batch, num_q_heads, hkv, D, max_pages_per_seq, sparse ? budget : 0);
     if (workspace_bytes < w.total) return SLC_ERR_WORKSPACE;
-    DeviceInfo* dev;
-    if ((rc = device_info(&dev))) return rc;
+    const DeviceCfg* dev;
+    if ((rc = device_cfg(&dev))) return rc;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     if (scale <= 0.f) scale = 1.f / sqrtf((float)D);
-    int32_t* sel = selected_out ? selected_out : reinterpret_cast<int32_t*>(ws + w.selected);
-    cudaError_t e = cudaSuccess;
     AttendParams ap{};
     ap.q = q;
     ap.k_cache = cache->k_cache;
     ap.v_cache = cache->v_cache;
     ap.block_table = block_table;
     ap.seq_lens = seq_lens;
-    ap.selected = sel;
     ap.part_acc = reinterpret_cast<float*>(ws + w.part_acc);
     ap.part_ml = reinterpret_cast<float2*>(ws + w.part_ml);
     ap.out = out;
@@ -249,35 +280,47 @@ static int decode(int mode, const void* q, const slc_cache_t* cache,
     ap.group = num_q_heads / hkv;
     ap.max_pages = max_pages_per_seq;
     ap.num_pages = cache->num_pages;
-    ap.list = sparse ? kListSparse : kListDense;
-    ap.prefix = prefix;
-    ap.window = window;
-    ap.budget = sparse ? budget : 0;
+    ap.prefix = sparse ? prefix : 0;
+    ap.window = sparse ? window : 0;
     ap.scale_log2 = scale * 1.4426950408889634f;
-    if (mode == 1 && budget > 0) {
-        // score -> select; the attention then waits for the selection
-        float* scores = reinterpret_cast<float*>(ws + w.scores);
-        const int cs = cand_stride_of(max_pages_per_seq);
-        ScoreParams sp{q,           cache->meta, block_table, seq_lens,
-                       scores,      dev->status, batch,
-                       num_q_heads, hkv,         num_q_heads / hkv, max_pages_per_seq,
-                       cache->num_pages, prefix, window, cs};
-        SelectParams lp{scores, seq_lens, sel,    dev->status, batch, hkv,
-                        max_pages_per_seq, prefix, window, budget, cs};
-        if (stage == 0 || stage == 1) {
-            e = launch_score(sp, D, dev->num_sms, stream);
-            if (e != cudaSuccess) return note_cuda(e, "score_pages");
-        }
-        if (stage == 0 || stage == 2) {
-            e = launch_select(lp, stream);
-            if (e != cudaSuccess) return note_cuda(e, "select_pages");
-        }
-        ap.wait_first = 1;
+    cudaError_t e;
+    if (!sparse) {
+        e = launch_dense(ap, D, *dev, stream);
+        return e == cudaSuccess ? SLC_OK : note_cuda(e, "dense");
     }
-    const int what = stage == 3 ? kAttendOnly : stage == 4 ? kMergeOnly : kAttendAndMerge;
-    if (stage == 1 || stage == 2) return SLC_OK;
-    e = launch_attend(ap, D, dev->num_sms, stream, what);
-    return e == cudaSuccess ? SLC_OK : note_cuda(e, "attend/merge");
+    const bool scoring = mode == 1 && budget > 0;
+    const int cs = cand_stride_of(max_pages_per_seq);
+    float* scores = reinterpret_cast<float*>(ws + w.scores);
+    StreamParams sp{};
+    sp.at = ap;
+    uint32_t* tile_max = reinterpret_cast<uint32_t*>(ws + w.tile_max);
+    sp.sc = ScoreParams{q,           cache->meta, block_table, seq_lens,
+                        scoring ? scores : nullptr, dev->status, batch,
+                        num_q_heads, hkv,         num_q_heads / hkv, max_pages_per_seq,
+                        cache->num_pages, prefix, window, cs, tile_max};
+    if (stage == 0 || stage == 1) {
+        e = launch_stream(sp, D, *dev, stream);
+        if (e != cudaSuccess) return note_cuda(e, "stream");
+        if (stage == 1) return SLC_OK;
+    } else {
+        // the finishing kernel alone: the streaming kernel's chunk count
+        sp.at.num_chunks = stream_chunks(D, *dev);
+        sp.at.list = kListForced;
+    }
+    FinishParams fp{};
+    fp.at = sp.at;
+    fp.scores = mode == 1 ? scores : nullptr;
+    fp.tile_max = tile_max;
+    fp.given = mode == 2 ? selected_out : nullptr;
+    fp.selected = mode == 1
+                      ? (selected_out ? selected_out : reinterpret_cast<int32_t*>(ws + w.selected))
+                      : nullptr;
+    fp.sel_phys = reinterpret_cast<int32_t*>(ws + w.sel_phys);
+    fp.budget = budget;
+    fp.cand_stride = cs;
+    fp.stream_scored = scoring ? 1 : 0;
+    e = launch_finish(fp, D, *dev, stream);
+    return e == cudaSuccess ? SLC_OK : note_cuda(e, "finish");
 }
 
 int slc_sparse_decode(const void* q, const slc_cache_t* cache, const int32_t* block_table,
@@ -296,7 +339,7 @@ int slc_sparse_decode_stage(int32_t stage, const void* q, const slc_cache_t* cac
                             int32_t prefix, int32_t window, int32_t budget, float scale,
                             float* out, int32_t* selected_out, void* workspace,
                             size_t workspace_bytes, slc_stream_t stream) {
-    if (stage < 1 || stage > 4) return SLC_ERR_INVALID_ARG;
+    if (stage < 1 || stage > 2) return SLC_ERR_INVALID_ARG;
     return decode(1, q, cache, block_table, max_pages_per_seq, seq_lens, batch, num_q_heads,
                   prefix, window, budget, scale, out, selected_out, workspace, workspace_bytes,
                   stream, stage);
@@ -354,15 +397,14 @@ int slc_sparse_decode_static(const void* q, const slc_cache_t* cache, const int3
                              int32_t num_q_heads, int32_t prefix, int32_t window, int32_t budget,
                              float scale, float* out, int32_t* selected_out,
                              slc_stream_t stream) {
-    int rc = check_cache(cache);
-    if (rc) return rc;
-    if ((rc = check_heads(cache, num_q_heads))) return rc;
-    if (batch < 0 || max_pages_per_seq <= 0 || budget < 0) return SLC_ERR_INVALID_ARG;
+    bool empty;
+    int rc = check_decode(1, q, cache, block_table, max_pages_per_seq, seq_lens, batch,
+                          num_q_heads, prefix, window, budget, scale, out, selected_out, &empty);
+    if (rc || empty) return rc;
     const size_t need = workspace_layout(batch, num_q_heads, cache->num_kv_heads,
                                          cache->head_dim, max_pages_per_seq, budget)
                             .total;
     if (need > SLC_STATIC_SCRATCH_BYTES) return SLC_ERR_WORKSPACE;
-    if (batch == 0) return SLC_OK;
     void* scratch = nullptr;
     if ((rc = static_scratch(&scratch))) return rc;
     return slc_sparse_decode(q, cache, block_table, max_pages_per_seq, seq_lens, batch,
@@ -372,9 +414,9 @@ int slc_sparse_decode_static(const void* q, const slc_cache_t* cache, const int3
 
 int slc_device_status(int32_t* status, slc_stream_t stream) {
     if (!status) return SLC_ERR_INVALID_ARG;
-    DeviceInfo* dev;
+    const DeviceCfg* dev;
     int rc;
-    if ((rc = device_info(&dev))) return rc;
+    if ((rc = device_cfg(&dev))) return rc;
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return note_cuda(e);
     unsigned v = 0;

@@ -6,9 +6,12 @@
 //           "Hybrid LLM Decoding 2.2x Faster at 256k, No Retraining",
 //           section "The remaining full-attention layers are the
 //           long-context bill")
-//   sparse  prefix pages, then the selected pages, then window pages
-//           (same article, section "The method: sliding window + prefix +
-//           query-aware pages, searched per layer")
+//   forced  prefix pages, then window pages (the part of the sparse step
+//           that needs no selection; same article, section "The method:
+//           sliding window + prefix + query-aware pages, searched per
+//           layer"), attended by the streaming kernel (slc_stream.cu)
+// This file holds the dense kernel and the merge; the per-warp attention is
+// in slc_attend_impl.cuh.
 // The lists of all units are concatenated and cut into equal chunks, one per
 // CTA of a persistent grid, so work is balanced by pages whatever the
 // sequence lengths.  A chunk that spans unit boundaries yields one partial
@@ -40,47 +43,13 @@ namespace {
 
 using namespace attn;
 
-// L2 prefetch of the K and V tiles of the prefix and window pages among
-// list positions [s, e) (sparse lists; every thread of the CTA calls it).
-template <int D>
-__device__ void prefetch_forced(const AttendParams& p, long long s, long long e) {
-    constexpr uint32_t TILE = kPage * D * 2;
-    if (s >= e) return;
-    auto len_of = [&](int b) { return list_len(p, b); };
-    int u;
-    long long ustart;
-    locate_unit(s, p.batch, p.hkv, len_of, &u, &ustart);  // warp-wide: every warp does it
-    while (s < e && u < p.batch * p.hkv) {
-        const int b = u / p.hkv, h = u % p.hkv;
-        const int len = list_len(p, b);
-        const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
-        const PageRanges r = page_ranges(L, p.prefix, p.window);
-        const int nforced = r.np + (r.n - r.ws);
-        const int i0 = (int)(s - ustart);
-        const int i1 = (int)(min(e, ustart + len) - ustart);
-        for (int i = i0 + (int)threadIdx.x; i < min(i1, nforced); i += blockDim.x) {
-            const int j = i < r.np ? i : r.ws + (i - r.np);
-            const int ph = p.block_table[(long long)b * p.max_pages + j];
-            if (ph >= 0 && ph < p.num_pages) {
-                const long long off = ((long long)ph * p.hkv + h) * TILE;
-                prefetch_l2(static_cast<const uint8_t*>(p.k_cache) + off, TILE);
-                prefetch_l2(static_cast<const uint8_t*>(p.v_cache) + off, TILE);
-            }
-        }
-        s = ustart + len;
-        ustart = s;
-        ++u;
-    }
-}
-
 // One CTA per chunk of the concatenated page lists.  For every unit piece
 // of the chunk, the CTA's warps take its pages round-robin, then combine
 // their partials in shared memory (reusing their rings) into one partial,
 // stored in slot (unit + chunk).
-// Residency: three CTAs per SM at d = 128 (64 KB of rings each), one at
-// d = 256; the register budget follows.
 template <int D, int NW, int STAGES>
-__global__ void __launch_bounds__(NW * 32, D == 128 ? 3 : 1) attend_kernel(AttendParams p) {
+__global__ void __launch_bounds__(NW * 32, (D == 128 && NW == 4) ? 3 : 1)
+    attend_kernel(AttendParams p) {
     constexpr int TILE = kPage * D * 2;
     constexpr int RING = STAGES * 2 * TILE;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -101,11 +70,8 @@ __global__ void __launch_bounds__(NW * 32, D == 128 ? 3 : 1) attend_kernel(Atten
     const long long cpp = (total + gridDim.x - 1) / gridDim.x;
     const long long s = (long long)blockIdx.x * cpp;
     const long long e = min(total, s + cpp);
-    // After a selection kernel: while it runs, only bring this chunk's
-    // prefix and window pages (known without the selection) into L2.  Every
-    // read of data waits for the preceding kernel (which may be writing the
-    // selection, the cache, or reading the partial slots).
-    if (p.wait_first) prefetch_forced<D>(p, s, e);
+    // every read of data waits for the preceding kernel (which may be writing
+    // the cache, or reading the partial slots)
     grid_dep_wait();
     uint32_t it = 0;
     bool ok = true;
@@ -122,7 +88,7 @@ template <int D>
 __global__ void __launch_bounds__(kMergeGroups * D / 4) merge_kernel(AttendParams p) {
     constexpr int V4 = D / 4;
     const int u = blockIdx.x, g = blockIdx.y;
-    const int b = u / p.hkv, h = u % p.hkv;
+    const int b = u / p.hkv;
     const int G = p.group;
     const int tid = threadIdx.x;
     const int grp = tid / V4, d4 = tid % V4;
@@ -133,22 +99,15 @@ __global__ void __launch_bounds__(kMergeGroups * D / 4) merge_kernel(AttendParam
     if (tid < 32) {
         auto len_of = [&](int bb) { return list_len(p, bb); };
         const long long total = total_units(p.batch, p.hkv, len_of);
-        long long base = 0;
-        for (int b0 = 0; b0 < b; b0 += 32) {
-            const int bb = b0 + tid;
-            long long c = bb < b ? (long long)list_len(p, bb) * p.hkv : 0;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-            base += c;
-        }
+        const long long base = unit_list_start(p, u);
         if (tid == 0) {
-            sh_off = base + (long long)h * list_len(p, b);
+            sh_off = base;
             sh_total = total;
         }
     }
     __syncthreads();
     const int len = list_len(p, b);
-    float* outp = p.out + ((long long)b * p.hq + h * G + g) * D;
+    float* outp = p.out + ((long long)b * p.hq + (u % p.hkv) * G + g) * D;
     if (len == 0) {
         grid_dep_wait();
         if (grp == 0) reinterpret_cast<float4*>(outp)[d4] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -166,21 +125,7 @@ __global__ void __launch_bounds__(kMergeGroups * D / 4) merge_kernel(AttendParam
         const float2 ml = __ldg(&p.part_ml[(u + k) * G + g]);
         const float4 a =
             __ldg(reinterpret_cast<const float4*>(p.part_acc + ((u + k) * G + g) * D) + d4);
-        if (ml.x > M) {  // new maximum: rescale what was summed so far
-            const float c = ex2(M - ml.x);
-            num.x *= c;
-            num.y *= c;
-            num.z *= c;
-            num.w *= c;
-            den *= c;
-            M = ml.x;
-        }
-        const float w = ml.x == -INFINITY ? 0.f : ex2(ml.x - M);  // empty partial
-        num.x = fmaf(w, a.x, num.x);
-        num.y = fmaf(w, a.y, num.y);
-        num.z = fmaf(w, a.z, num.z);
-        num.w = fmaf(w, a.w, num.w);
-        den = fmaf(w, ml.y, den);
+        fold_partial(ml, a, M, num, den);
     }
     sh_num[grp][d4] = num;
     if (d4 == 0) {
@@ -216,49 +161,49 @@ constexpr int attend_smem() {
     return NW * STAGES * (2 * kPage * D * 2 + 8 + 4);
 }
 
-// CTAs (chunks) of an attention launch: all that fit on the GPU at once,
-// at most kMaxAttendChunks.
 template <int D, int NW, int STAGES>
-cudaError_t grid_of(int num_sms, int* blocks) {
+cudaError_t setup_one(int* occ) {
     constexpr int smem = attend_smem<D, NW, STAGES>();
-    static int occ = 0;
-    if (occ == 0) {
-        cudaError_t e = cudaFuncSetAttribute(attend_kernel<D, NW, STAGES>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, attend_kernel<D, NW, STAGES>,
-                                                          NW * 32, smem);
-        if (e != cudaSuccess) return e;
-        if (occ < 1) occ = 1;
-    }
-    *blocks = num_sms * occ;
-    if (*blocks > kMaxAttendChunks) *blocks = kMaxAttendChunks;
+    cudaError_t e = cudaFuncSetAttribute(attend_kernel<D, NW, STAGES>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, attend_kernel<D, NW, STAGES>,
+                                                      NW * 32, smem);
+    if (e != cudaSuccess) return e;
+    if (*occ < 1) *occ = 1;
     return cudaSuccess;
 }
 
+// One CTA (chunk) per resident slot of the GPU, at most kMaxAttendChunks.
 template <int D, int NW, int STAGES>
-cudaError_t run(AttendParams p, int num_sms, cudaStream_t stream, int what) {
+cudaError_t run(AttendParams p, int occ, int num_sms, cudaStream_t stream) {
     constexpr int smem = attend_smem<D, NW, STAGES>();
-    int blocks = 0;
-    cudaError_t e = grid_of<D, NW, STAGES>(num_sms, &blocks);
+    int blocks = num_sms * occ;
+    if (blocks > kMaxAttendChunks) blocks = kMaxAttendChunks;
+    p.num_chunks = blocks;
+    cudaError_t e = launch_pdl(attend_kernel<D, NW, STAGES>, dim3(blocks), dim3(NW * 32), smem,
+                               stream, 1, p);
     if (e != cudaSuccess) return e;
-    p.num_chunks = blocks;  // chunk count (one chunk per CTA)
-    if (what != kMergeOnly)
-        e = launch_pdl(attend_kernel<D, NW, STAGES>, dim3(blocks), dim3(NW * 32), smem, stream,
-                       p);
-    if (e != cudaSuccess || what == kAttendOnly) return e;
     return launch_pdl(merge_kernel<D>, dim3(p.batch * p.hkv, p.group),
-                      dim3(kMergeGroups * D / 4), 0, stream, p);
+                      dim3(kMergeGroups * D / 4), 0, stream, 1, p);
 }
 
 }  // namespace
 
-cudaError_t launch_attend(AttendParams p, int head_dim, int num_sms, cudaStream_t stream,
-                          int what) {
+// The dense list streams every page: at d = 128 one 8-warp CTA per SM with
+// two ring stages per warp keeps the most bytes in flight.
+cudaError_t setup_attend(DeviceCfg& d) {
+    cudaError_t e = setup_one<128, 8, 2>(&d.occ_attend[1]);
+    if (e == cudaSuccess) e = setup_one<256, 4, 3>(&d.occ_attend[2]);
+    d.occ_attend[0] = 0;
+    return e;
+}
+
+cudaError_t launch_dense(AttendParams p, int head_dim, const DeviceCfg& d, cudaStream_t stream) {
     if (p.batch * p.hkv == 0) return cudaSuccess;
-    // D=128: 4 warps x 2 stages x 8 KB = 64 KB per CTA, three CTAs per SM
-    if (head_dim == 128) return run<128, 4, 2>(p, num_sms, stream, what);
-    return run<256, 4, 3>(p, num_sms, stream, what);
+    p.list = kListDense;
+    if (head_dim == 128) return run<128, 8, 2>(p, d.occ_attend[1], d.num_sms, stream);
+    return run<256, 4, 3>(p, d.occ_attend[2], d.num_sms, stream);
 }
 
 }  // namespace slc

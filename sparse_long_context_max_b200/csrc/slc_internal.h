@@ -13,25 +13,56 @@ namespace slc {
 // Launch with programmatic stream serialization: the kernel may start while
 // the preceding kernel in the stream is still running; it calls
 // grid_dep_wait() before touching anything that kernel produces.
+// cluster > 1 also sets the thread-block cluster size (x).
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t stream, Args&&... args) {
+                       cudaStream_t stream, int cluster, Args&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    int n = 1;
+    if (cluster > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = cluster;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        n = 2;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = n;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Upper bound on the number of attention CTAs (chunks) of one launch; sizes
 // the split-partial workspace (slot = unit + chunk index).
 constexpr int kMaxAttendChunks = 1024;
+
+// Cluster sizes the finishing kernel may be launched with.
+constexpr int kFinishClusters[] = {16, 8};
+constexpr int kNumFinishClusters = 2;
+
+// Per-device launch settings, looked up once per device (with that device
+// current) by slc_api.cu and passed to every launch.
+struct DeviceCfg {
+    int device;
+    int num_sms;
+    unsigned* status;  // the device status word
+    int occ_score[2];       // score_kernel CTAs per SM (D = 128, 256)
+    int occ_stream[2];      // stream_kernel CTAs per SM (D = 128, 256)
+    int occ_attend[3];      // attend_kernel CTAs per SM (D = 128 sparse shape, D = 128 dense, D = 256)
+    int finish_clusters[2][kNumFinishClusters];  // co-resident finish clusters (D, cluster size)
+};
+
+cudaError_t setup_score(DeviceCfg& d);
+cudaError_t setup_select(DeviceCfg& d);
+cudaError_t setup_attend(DeviceCfg& d);
+cudaError_t setup_stream(DeviceCfg& d);
+cudaError_t setup_finish(DeviceCfg& d);
 
 struct KvAppendParams {
     const void* k_new;
@@ -63,6 +94,9 @@ struct ScoreParams {
     unsigned* status;
     int batch, hq, hkv, group, max_pages, num_pages, prefix, window;
     int cand_stride;  // 0: scores indexed by page; else rows of cand_stride by candidate
+    // (rows by candidate only, nullable) the largest order key (see
+    // order_key) of each 16-candidate tile: [units][cand_stride / 16]
+    uint32_t* tile_max;
 };
 
 struct SelectParams {
@@ -80,7 +114,7 @@ constexpr int kSelTile = 16;
 inline int cand_stride_of(int max_pages) { return (max_pages + 63) / 64 * 64; }
 
 // Page list attended per unit (see slc_attend_impl.cuh).
-enum : int { kListDense = 0, kListSparse = 1 };
+enum : int { kListDense = 0, kListForced = 1 };
 
 struct AttendParams {
     const void* q;
@@ -88,22 +122,44 @@ struct AttendParams {
     const void* v_cache;
     const int32_t* block_table;
     const int32_t* seq_lens;
-    const int32_t* selected;  // sparse only: [B][Hkv][budget]
     float* part_acc;          // [slots][group][D]
     float2* part_ml;          // [slots][group]  (running max in log2 units, sum)
     float* out;               // [B][Hq][D]
     unsigned* status;
     int batch, hq, hkv, group, max_pages, num_pages;
-    int list;  // kListDense or kListSparse
-    int prefix, window, budget;
+    int list;  // kListDense or kListForced
+    int prefix, window;
     float scale_log2;  // softmax scale * log2(e)
     int num_chunks;    // chunks of the attention launch (one per CTA)
-    int wait_first;    // the preceding kernel writes the selection: L2-prefetch the forced pages first
+};
+
+// The streaming kernel: per unit, attention over the prefix and window pages
+// (split partials, as attend_kernel with kListForced) and, unless
+// score.scores is null, the scores of the candidate pages (as score_kernel,
+// rows by candidate).
+struct StreamParams {
+    AttendParams at;
+    ScoreParams sc;
+};
+
+// The finishing kernel: per unit, the selection (from the scores, or given),
+// attention over the selected pages, and the merge of those partials with
+// the streaming kernel's prefix/window partials into out.
+struct FinishParams {
+    AttendParams at;        // at.part_acc / at.part_ml: the streaming kernel's partials;
+                            // at.num_chunks: the streaming kernel's grid
+    int stream_scored;      // the streaming kernel scored (its grid split, forced_ctas)
+    const float* scores;    // [units][cand_stride] by candidate, or null (selection given)
+    const uint32_t* tile_max;  // [units][cand_stride / 16] tile maxima (order keys)
+    const int32_t* given;   // [units][budget] given selection (scores == null)
+    int32_t* selected;      // [units][budget] out: ascending, -1 padded (scores != null)
+    int32_t* sel_phys;      // [units][budget] workspace: physical page of each selected entry
+    int budget, cand_stride;
 };
 
 // Workspace carve-up shared by the API and the size query.
 struct WorkspaceLayout {
-    size_t scores, selected, part_acc, part_ml, total;
+    size_t scores, tile_max, selected, sel_phys, part_acc, part_ml, total;
 };
 
 // Split-partial slots of an attention launch: unit + chunk, chunks <=
@@ -111,15 +167,19 @@ struct WorkspaceLayout {
 inline size_t partial_slots(size_t units) { return units + kMaxAttendChunks; }
 
 cudaError_t launch_kv_append(const KvAppendParams& p, int head_dim, cudaStream_t stream);
-cudaError_t launch_build_meta(const BuildMetaParams& p, int head_dim, int num_sms,
+cudaError_t launch_build_meta(const BuildMetaParams& p, int head_dim, const DeviceCfg& d,
                               cudaStream_t stream);
-cudaError_t launch_score(const ScoreParams& p, int head_dim, int num_sms, cudaStream_t stream);
+cudaError_t launch_score(const ScoreParams& p, int head_dim, const DeviceCfg& d,
+                         cudaStream_t stream);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
-// Attention over the list of each unit (dense: all pages; sparse: prefix,
-// window, selected), then the merge of the split partials into out.  what:
-// kAttendAndMerge, or one of the two kernels alone (for stage timing).
-enum : int { kAttendAndMerge = 0, kAttendOnly = 1, kMergeOnly = 2 };
-cudaError_t launch_attend(AttendParams p, int head_dim, int num_sms, cudaStream_t stream,
-                          int what = kAttendAndMerge);
+// Dense attention over every page of every unit, then the merge of the split
+// partials into out.
+cudaError_t launch_dense(AttendParams p, int head_dim, const DeviceCfg& d, cudaStream_t stream);
+// The streaming kernel; sets p.at.num_chunks to its grid size
+// (stream_chunks) and p.at.list to kListForced.
+cudaError_t launch_stream(StreamParams& p, int head_dim, const DeviceCfg& d, cudaStream_t stream);
+int stream_chunks(int head_dim, const DeviceCfg& d);
+// The finishing kernel (p.at.num_chunks: the streaming kernel's grid).
+cudaError_t launch_finish(FinishParams p, int head_dim, const DeviceCfg& d, cudaStream_t stream);
 
 }  // namespace slc

@@ -146,12 +146,13 @@ cudaError_t launch_kv_append(const KvAppendParams& p, int head_dim, cudaStream_t
     const int threads = 128;
     const int blocks = (warps * 32 + threads - 1) / threads;
     if (head_dim == 128)
-        return launch_pdl(kv_append_kernel<128>, dim3(blocks), dim3(threads), 0, stream, p);
-    return launch_pdl(kv_append_kernel<256>, dim3(blocks), dim3(threads), 0, stream, p);
+        return launch_pdl(kv_append_kernel<128>, dim3(blocks), dim3(threads), 0, stream, 1, p);
+    return launch_pdl(kv_append_kernel<256>, dim3(blocks), dim3(threads), 0, stream, 1, p);
 }
 
-cudaError_t launch_build_meta(const BuildMetaParams& p, int head_dim, int num_sms,
+cudaError_t launch_build_meta(const BuildMetaParams& p, int head_dim, const DeviceCfg& d,
                               cudaStream_t stream) {
+    const int num_sms = d.num_sms;
     const long long tasks = (long long)p.batch * p.max_pages * p.hkv;
     const int threads = 256;
     long long blocks = (tasks * 32 + threads - 1) / threads;

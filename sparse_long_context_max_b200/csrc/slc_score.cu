@@ -7,12 +7,13 @@
 //
 // Work split: tiles (16 consecutive candidate pages of one unit) of all
 // units are numbered in (b, h, tile) order and every warp of the
-// (persistent) grid takes a contiguous range of them.  Each warp streams
-// its tiles through a private shared-memory ring (two 8 KB tiles at D=128)
-// filled by 16-byte asynchronous copies, one cp.async group per tile.
-// Three 4-warp CTAs per SM keep 24 tiles (192 KB) in flight.  The kernel
-// also writes each tile's maximum score when asked, which the selection
-// uses to discard most pages without reading their scores.
+// (persistent) grid takes a contiguous range of them (score_range in
+// slc_score_impl.cuh).  Each warp streams its tiles through a private
+// shared-memory ring (two 8 KB tiles at D=128) filled by 16-byte
+// asynchronous copies, one cp.async group per tile.  Three 4-warp CTAs per
+// SM keep 24 tiles (192 KB) in flight.  The streaming kernel
+// (slc_stream.cu) runs the same range code after its prefix/window
+// attention.
 #include "slc_score_impl.cuh"
 
 namespace slc {
@@ -30,122 +31,48 @@ struct ScoreCfg : TileGeom<D> {
     static constexpr int SMEM = kScoreWarps * RING_B;  // 64 KB: three CTAs per SM
 };
 
-// Cursor over the tiles of consecutive units.
-struct TileCursor {
-    int u;
-    int ustart;  // global index of the unit's first tile
-    int ntiles;  // tiles of unit u
-    PageRanges r;
-};
-
-__device__ __forceinline__ void cursor_seek(const ScoreParams& p, TileCursor& c, int g) {
-    while (true) {
-        const int L = checked_len(p.seq_lens, c.u / p.hkv, p.max_pages, p.status);
-        c.r = page_ranges(L, p.prefix, p.window);
-        c.ntiles = (c.r.ws - c.r.np + kTilePages - 1) / kTilePages;
-        if (g - c.ustart < c.ntiles) return;
-        c.ustart += c.ntiles;
-        ++c.u;
-    }
-}
-
 template <int D>
 __global__ void __launch_bounds__(kScoreWarps * 32, 3) score_kernel(ScoreParams p) {
     using C = ScoreCfg<D>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
-    uint8_t* ring = smem + warp * C::RING_B;
-
     // inputs (q, metadata, lengths) may come from the preceding kernel
     grid_dep_wait();
     grid_dep_launch();
-
-    const int gw = blockIdx.x * kScoreWarps + warp;
-    const int nw = gridDim.x * kScoreWarps;
-    auto tiles_of = [&](int b) {
-        const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
-        const PageRanges r = page_ranges(L, p.prefix, p.window);
-        return (r.ws - r.np + kTilePages - 1) / kTilePages;
-    };
-    const int total = (int)total_units(p.batch, p.hkv, tiles_of);
-    const int per = (total + nw - 1) / nw;
-    const int g0 = gw * per;
-    const int g_end = min(total, g0 + per);
-    if (g0 >= g_end) return;
-
-    TileCursor use, iss;
-    {
-        long long us;
-        locate_unit(g0, p.batch, p.hkv, tiles_of, &use.u, &us);
-        use.ustart = (int)us;
-    }
-    cursor_seek(p, use, g0);
-    iss = use;
-    // issue side: tile gi is the next to copy; pf holds its page ids, loaded
-    // one copy ahead so the lookup overlaps the ring traffic.  Every call
-    // commits exactly one group (possibly empty) so that wait_group<NT-1>
-    // always means "the oldest tile has landed".
-    int gi = g0;
-    int pf = tile_phys(p, iss.u, iss.r, gi - iss.ustart);
-    auto copy_next = [&](int slot) {
-        if (gi < g_end) {
-            copy_tile<D>(p, iss.u % p.hkv, pf, ring + slot * C::TILE_B);
-            ++gi;
-            if (gi < g_end) {
-                if (gi - iss.ustart >= iss.ntiles) cursor_seek(p, iss, gi);
-                pf = tile_phys(p, iss.u, iss.r, gi - iss.ustart);
-            }
-        } else {
-            cp_async_commit();
-        }
-    };
-#pragma unroll
-    for (int k = 0; k < C::NT; ++k) copy_next(k);
-
-    int wu = -1;  // unit whose weights are loaded
-    float w[C::CPL][8];
-    for (int g = g0; g < g_end; ++g) {
-        if (g - use.ustart >= use.ntiles) cursor_seek(p, use, g);
-        if (use.u != wu) {
-            wu = use.u;
-            load_weights<D>(p, use.u, w);
-        }
-        const int slot = (g - g0) % C::NT;
-        cp_async_wait<C::NT - 1>();  // this lane's chunks of the tile have landed
-        score_tile<D>(p, use.u, use.r, g - use.ustart, ring + slot * C::TILE_B, w);
-        copy_next(slot);  // refill: this lane's reads of the slot are done
-    }
-    cp_async_wait<0>();
+    score_range<D, C::NT>(p, smem + warp * C::RING_B, blockIdx.x * kScoreWarps + warp,
+                          gridDim.x * kScoreWarps);
 }
 
 }  // namespace
 
-cudaError_t launch_score(const ScoreParams& p, int head_dim, int num_sms, cudaStream_t stream) {
-    static int occ128 = 0, occ256 = 0;
-    int& occ = head_dim == 128 ? occ128 : occ256;
-    const int smem = head_dim == 128 ? ScoreCfg<128>::SMEM : ScoreCfg<256>::SMEM;
-    if (occ == 0) {
-        cudaError_t e;
-        if (head_dim == 128) {
-            e = cudaFuncSetAttribute(score_kernel<128>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (e == cudaSuccess)
-                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, score_kernel<128>,
-                                                                  kScoreWarps * 32, smem);
-        } else {
-            e = cudaFuncSetAttribute(score_kernel<256>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (e == cudaSuccess)
-                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, score_kernel<256>,
-                                                                  kScoreWarps * 32, smem);
-        }
-        if (e != cudaSuccess) return e;
-        if (occ < 1) occ = 1;
-    }
-    const int blocks = num_sms * occ;
-    if (head_dim == 128)
-        return launch_pdl(score_kernel<128>, dim3(blocks), dim3(kScoreWarps * 32), smem, stream, p);
-    return launch_pdl(score_kernel<256>, dim3(blocks), dim3(kScoreWarps * 32), smem, stream, p);
+cudaError_t setup_score(DeviceCfg& d) {
+    const int smem128 = ScoreCfg<128>::SMEM, smem256 = ScoreCfg<256>::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(score_kernel<128>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem128);
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_score[0], score_kernel<128>,
+                                                          kScoreWarps * 32, smem128);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(score_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem256);
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_score[1], score_kernel<256>,
+                                                          kScoreWarps * 32, smem256);
+    for (int i = 0; i < 2; ++i)
+        if (d.occ_score[i] < 1) d.occ_score[i] = 1;
+    return e;
+}
+
+cudaError_t launch_score(const ScoreParams& p, int head_dim, const DeviceCfg& d,
+                         cudaStream_t stream) {
+    const bool d128 = head_dim == 128;
+    const int smem = d128 ? ScoreCfg<128>::SMEM : ScoreCfg<256>::SMEM;
+    const int blocks = d.num_sms * d.occ_score[d128 ? 0 : 1];
+    if (d128)
+        return launch_pdl(score_kernel<128>, dim3(blocks), dim3(kScoreWarps * 32), smem, stream,
+                          1, p);
+    return launch_pdl(score_kernel<256>, dim3(blocks), dim3(kScoreWarps * 32), smem, stream, 1,
+                      p);
 }
 
 }  // namespace slc

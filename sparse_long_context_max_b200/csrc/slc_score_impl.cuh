@@ -125,11 +125,12 @@ __device__ __forceinline__ void copy_tile(const ScoreParams& p, int h, int phys,
 }
 
 // Score the landed tile jt of unit u (rows in `tile`) and write the page
-// scores.
+// scores; lane i < 16 holds page i's physical page in tphys (-1: the
+// block-table entry failed its check, and the page scores -inf).
 template <int D>
 __device__ __forceinline__ void score_tile(const ScoreParams& p, int u, const PageRanges& r,
                                            int jt, const uint8_t* tile,
-                                           const float (&w)[TileGeom<D>::CPL][8]) {
+                                           const float (&w)[TileGeom<D>::CPL][8], int tphys) {
     using C = TileGeom<D>;
     const int lane = threadIdx.x & 31;
     const uint8_t* t = tile + lane * 16;
@@ -157,15 +158,203 @@ __device__ __forceinline__ void score_tile(const ScoreParams& p, int u, const Pa
     }
     acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
     const int j = r.np + jt * kTilePages + (lane >> 1);
+    const int phys = __shfl_sync(0xffffffffu, tphys, lane >> 1);
+    // a page whose block-table entry failed its check scores -inf
+    const float sc = phys < 0 ? -INFINITY : acc[0];
     if (j < r.ws && (lane & 1) == 0) {
-        // a page whose block-table entry failed its check scores -inf
-        const int phys = p.block_table[(long long)(u / p.hkv) * p.max_pages + j];
-        const float sc = (phys < 0 || phys >= p.num_pages) ? -INFINITY : acc[0];
         if (p.cand_stride)
             p.scores[(long long)u * p.cand_stride + (j - r.np)] = sc;
         else
             p.scores[(long long)u * p.max_pages + j] = sc;
     }
+    if (p.tile_max) {  // the tile's largest key, over its candidates
+        const uint32_t m = __reduce_max_sync(0xffffffffu, j < r.ws ? order_key(sc) : 0u);
+        if (lane == 0) p.tile_max[(long long)u * (p.cand_stride / kTilePages) + jt] = m;
+    }
+}
+
+
+// Cursor over the tiles of consecutive units.
+struct TileCursor {
+    int u;
+    int ustart;  // global index of the unit's first tile
+    int ntiles;  // tiles of unit u
+    PageRanges r;
+};
+
+__device__ __forceinline__ void cursor_seek(const ScoreParams& p, TileCursor& c, int g) {
+    while (true) {
+        const int L = checked_len(p.seq_lens, c.u / p.hkv, p.max_pages, p.status);
+        c.r = page_ranges(L, p.prefix, p.window);
+        c.ntiles = (c.r.ws - c.r.np + kTilePages - 1) / kTilePages;
+        if (g - c.ustart < c.ntiles) return;
+        c.ustart += c.ntiles;
+        ++c.u;
+    }
+}
+
+// Score the tiles of warp gw of nw (tiles of all units numbered in (b, h,
+// tile) order, a contiguous range per warp) through this warp's ring of NT
+// tiles at `ring` (NT * TILE_B bytes).  The caller has waited for the
+// kernel that produces q, the metadata or the lengths.
+template <int D, int NT>
+__device__ void score_range(const ScoreParams& p, uint8_t* ring, int gw, int nw) {
+    using C = TileGeom<D>;
+    auto tiles_of = [&](int b) {
+        const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
+        const PageRanges r = page_ranges(L, p.prefix, p.window);
+        return (r.ws - r.np + kTilePages - 1) / kTilePages;
+    };
+    const int total = (int)total_units(p.batch, p.hkv, tiles_of);
+    const int per = (total + nw - 1) / nw;
+    const int g0 = gw * per;
+    const int g_end = min(total, g0 + per);
+    if (g0 >= g_end) return;
+
+    TileCursor use, iss;
+    {
+        long long us;
+        locate_unit(g0, p.batch, p.hkv, tiles_of, &use.u, &us);
+        use.ustart = (int)us;
+    }
+    cursor_seek(p, use, g0);
+    iss = use;
+    // issue side: tile gi is the next to copy; pf holds its page ids, loaded
+    // one copy ahead so the lookup overlaps the ring traffic.  Every call
+    // commits exactly one group (possibly empty) so that wait_group<NT-1>
+    // always means "the oldest tile has landed".
+    int gi = g0;
+    int pf = tile_phys(p, iss.u, iss.r, gi - iss.ustart);
+    int sp[NT];  // page ids of the tile in each slot (lane i: page i)
+    auto copy_next = [&](int slot) {
+        if (gi < g_end) {
+#pragma unroll
+            for (int k = 0; k < NT; ++k)
+                if (k == slot) sp[k] = pf;
+            copy_tile<D>(p, iss.u % p.hkv, pf, ring + slot * C::TILE_B);
+            ++gi;
+            if (gi < g_end) {
+                if (gi - iss.ustart >= iss.ntiles) cursor_seek(p, iss, gi);
+                pf = tile_phys(p, iss.u, iss.r, gi - iss.ustart);
+            }
+        } else {
+            cp_async_commit();
+        }
+    };
+#pragma unroll
+    for (int k = 0; k < NT; ++k) copy_next(k);
+
+    int wu = -1;  // unit whose weights are loaded
+    float w[C::CPL][8];
+    for (int g = g0; g < g_end; ++g) {
+        if (g - use.ustart >= use.ntiles) cursor_seek(p, use, g);
+        if (use.u != wu) {
+            wu = use.u;
+            load_weights<D>(p, use.u, w);
+        }
+        const int slot = (g - g0) % NT;
+        cp_async_wait<NT - 1>();  // this lane's chunks of the tile have landed
+        int tp = sp[0];
+#pragma unroll
+        for (int k = 1; k < NT; ++k)
+            if (k == slot) tp = sp[k];
+        score_tile<D>(p, use.u, use.r, g - use.ustart, ring + slot * C::TILE_B, w, tp);
+        copy_next(slot);  // refill: this lane's reads of the slot are done
+    }
+    cp_async_wait<0>();
+}
+
+// score_range with the tiles brought in by bulk copies (TMA engine, one per
+// page row of 4*D bytes, issued by lanes 0..15) completing on the ring
+// stage's mbarrier, instead of per-lane 16-byte copies: the streaming
+// kernel's form.  bars: NT mbarriers (count 1) whose next phase parity is
+// `it` (ring uses so far, advanced here).  A bounded wait that gives up sets
+// SLC_STATUS_WAIT_TIMEOUT; the warp then drains its copies and stops.
+template <int D, int NT>
+__device__ void score_range_bulk(const ScoreParams& p, uint8_t* ring, uint64_t* bars,
+                                 uint32_t& it, int gw, int nw) {
+    using C = TileGeom<D>;
+    const int lane = threadIdx.x & 31;
+    auto tiles_of = [&](int b) {
+        const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
+        const PageRanges r = page_ranges(L, p.prefix, p.window);
+        return (r.ws - r.np + kTilePages - 1) / kTilePages;
+    };
+    const int total = (int)total_units(p.batch, p.hkv, tiles_of);
+    const int per = (total + nw - 1) / nw;
+    const int g0 = gw * per;
+    const int g_end = min(total, g0 + per);
+    if (g0 >= g_end) return;
+
+    TileCursor use, iss;
+    {
+        long long us;
+        locate_unit(g0, p.batch, p.hkv, tiles_of, &use.u, &us);
+        use.ustart = (int)us;
+    }
+    cursor_seek(p, use, g0);
+    iss = use;
+    int gi = g0;
+    int pf = tile_phys(p, iss.u, iss.r, gi - iss.ustart);
+    int sp[NT];  // page ids of the tile in each slot (lane i: page i)
+    const uint8_t* meta = static_cast<const uint8_t*>(p.meta);
+    // issue tile gi into stage `slot` (page ids in pf), then look one tile ahead
+    auto copy_next = [&](int slot) {
+        if (gi >= g_end) return;
+#pragma unroll
+        for (int k = 0; k < NT; ++k)
+            if (k == slot) sp[k] = pf;
+        const unsigned have = __ballot_sync(0xffffffffu, pf >= 0);
+        if (lane == 0) {
+            if (have) mbar_arrive_expect_tx(bars + slot, __popc(have) * C::PAGE_B);
+            else mbar_arrive(bars + slot);
+        }
+        __syncwarp();
+        if (pf >= 0) {
+            const long long src = ((long long)pf * p.hkv + iss.u % p.hkv) * C::PAGE_B;
+            bulk_g2s(ring + slot * C::TILE_B + lane * C::PAGE_B, meta + src, C::PAGE_B,
+                     bars + slot);
+        }
+        ++gi;
+        if (gi < g_end) {
+            if (gi - iss.ustart >= iss.ntiles) cursor_seek(p, iss, gi);
+            pf = tile_phys(p, iss.u, iss.r, gi - iss.ustart);
+        }
+    };
+    fence_proxy_async_smem();  // earlier generic accesses of the ring first
+#pragma unroll
+    for (int k = 0; k < NT; ++k) copy_next((it + k) % NT);
+
+    int wu = -1;  // unit whose weights are loaded
+    float w[C::CPL][8];
+    for (int g = g0; g < g_end; ++g) {
+        if (g - use.ustart >= use.ntiles) cursor_seek(p, use, g);
+        if (use.u != wu) {
+            wu = use.u;
+            load_weights<D>(p, use.u, w);
+        }
+        const uint32_t u_ = it + (g - g0);
+        const int slot = u_ % NT;
+        if (!mbar_wait_bounded(bars + slot, (u_ / NT) & 1u, 1u << 22)) {
+            if (lane == 0) {
+                atomicOr(p.status, SLC_STATUS_WAIT_TIMEOUT);
+                for (int k = g + 1; k < g_end && k < g + NT; ++k) {
+                    const uint32_t u2 = it + (k - g0);
+                    mbar_wait_bounded(bars + u2 % NT, (u2 / NT) & 1u, 1u << 22);
+                }
+            }
+            __syncwarp();
+            return;
+        }
+        int tp = sp[0];
+#pragma unroll
+        for (int k = 1; k < NT; ++k)
+            if (k == slot) tp = sp[k];
+        score_tile<D>(p, use.u, use.r, g - use.ustart, ring + slot * C::TILE_B, w, tp);
+        fence_proxy_async_smem();  // this warp's reads of the slot precede its refill
+        copy_next(slot);
+    }
+    it += g_end - g0;
 }
 
 }  // namespace scr

@@ -33,19 +33,20 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(SelectParams p) {
 
 template <int KPT>
 cudaError_t launch(const SelectParams& p, cudaStream_t stream) {
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(select_kernel<KPT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             select_smem<KPT>());
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
     return launch_pdl(select_kernel<KPT>, dim3(p.batch * p.hkv), dim3(kThreads),
-                      select_smem<KPT>(), stream, p);
+                      select_smem<KPT>(), stream, 1, p);
 }
 
 }  // namespace
+
+cudaError_t setup_select(DeviceCfg&) {
+    cudaError_t e = cudaFuncSetAttribute(select_kernel<16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         select_smem<16>());
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(select_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                select_smem<32>());
+}
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
     if (p.batch * p.hkv == 0) return cudaSuccess;

@@ -32,11 +32,6 @@
 namespace slc {
 namespace sel {
 
-__device__ __forceinline__ uint32_t order_key(float f) {
-    if (f == 0.f) f = 0.f;  // -0 and +0 tie
-    const uint32_t u = __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 template <int NTHR>
 struct Scratch {
@@ -264,10 +259,18 @@ __device__ void select_unit(const SelectParams& p, int u, Scratch<NTHR>& sc, uin
         mbar_arrive_expect_tx(bar, bytes);
         bulk_g2s(stage, p.scores + (long long)u * p.cand_stride, bytes, bar);
     }
-    auto landed = [&]() {  // every thread; the copy must land before the CTA exits
-        __syncthreads();     // the barrier is initialised
-        if (!mbar_wait_bounded(bar, 0, 1u << 22) && tid == 0)
-            atomicOr(p.status, SLC_STATUS_WAIT_TIMEOUT);
+    // every thread; the copy must land before the CTA exits.  Returns false
+    // (for every thread) if any thread's bounded wait gave up: the unit's
+    // selection is then written as all -1 instead of from unlanded scores.
+    auto landed = [&]() -> bool {
+        __syncthreads();  // the barrier is initialised
+        const bool timed_out = !mbar_wait_bounded(bar, 0, 1u << 22);
+        if (__syncthreads_or(timed_out)) {
+            if (tid == 0) atomicOr(p.status, SLC_STATUS_WAIT_TIMEOUT);
+            mbar_wait_bounded(bar, 0, 1u << 22);  // drain the copy before leaving
+            return false;
+        }
+        return true;
     };
     const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
     const PageRanges r = page_ranges(L, p.prefix, p.window);
@@ -277,12 +280,12 @@ __device__ void select_unit(const SelectParams& p, int u, Scratch<NTHR>& sc, uin
 
     if (nsel >= ncand) {  // every candidate is kept (also covers ncand == 0)
         for (int i = tid; i < p.budget; i += NTHR) out[i] = i < ncand ? r.np + i : -1;
-        if (bulk) landed();
+        if (bulk) (void)landed();
         return;
     }
     for (int i = nsel + tid; i < p.budget; i += NTHR) out[i] = -1;
     if (nsel <= 0) {
-        if (bulk) landed();
+        if (bulk) (void)landed();
         return;
     }
 
@@ -291,7 +294,10 @@ __device__ void select_unit(const SelectParams& p, int u, Scratch<NTHR>& sc, uin
     const int n_t = max(0, min(KPT, ncand - c0));
     float f[KPT];
     if (bulk) {
-        landed();
+        if (!landed()) {
+            for (int i = tid; i < nsel; i += NTHR) out[i] = -1;
+            return;
+        }
         const float4* s4 = reinterpret_cast<const float4*>(stage + c0);
 #pragma unroll
         for (int q = 0; q < KPT / 4; ++q) {

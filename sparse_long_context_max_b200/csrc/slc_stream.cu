@@ -1,0 +1,117 @@
+// The streaming half of the sparse decode step: everything that does not
+// depend on the selection, in one persistent HBM-bound kernel over every SM.
+//
+//   - attention over each unit's prefix and window pages (the pages every
+//     query keeps: "Hybrid LLM Decoding 2.2x Faster at 256k, No
+//     Retraining", section "The method: sliding window + prefix +
+//     query-aware pages, searched per layer"), as split partials exactly
+//     like the dense kernel's (slot = unit + chunk, the forced lists of all
+//     units concatenated and cut into one chunk per attending CTA);
+//   - the Quest bound of every candidate page (same section), written by
+//     candidate into 16-byte aligned rows, as score_kernel does.
+//
+// The two run side by side: the first CTAs of the grid attend, the others
+// score, split in proportion to their bytes (forced_ctas in
+// slc_attend_impl.cuh; a K+V page stage and a 16-page metadata tile are
+// both 64*D bytes).  The finishing kernel (slc_finish.cu) then selects,
+// attends the selected pages and merges everything.
+#include "slc_attend_impl.cuh"
+#include "slc_score_impl.cuh"
+
+namespace slc {
+
+namespace {
+
+using namespace attn;
+
+template <int D>
+struct StreamCfg {
+    static constexpr int NW = 4;                   // warps per CTA
+    static constexpr int STAGES = D == 128 ? 2 : 3;  // ring stages per warp
+    static constexpr int RING = STAGES * 2 * kPage * D * 2;
+    static constexpr int SMEM = NW * STAGES * (2 * kPage * D * 2 + 8 + 4);
+    static constexpr int MIN_BLOCKS = D == 128 ? 3 : 1;
+};
+
+template <int D>
+__global__ void __launch_bounds__(StreamCfg<D>::NW * 32, StreamCfg<D>::MIN_BLOCKS)
+    stream_kernel(StreamParams p) {
+    using C = StreamCfg<D>;
+    static_assert(C::RING == C::STAGES * scr::TileGeom<D>::TILE_B, "ring holds NT tiles");
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    Ring ring;
+    ring.tiles = smem + warp * C::RING;
+    ring.bars = reinterpret_cast<uint64_t*>(smem + C::NW * C::RING) + warp * C::STAGES;
+    ring.nvalid =
+        reinterpret_cast<int*>(smem + C::NW * C::RING + C::NW * C::STAGES * 8) + warp * C::STAGES;
+    if (lane == 0) {
+        for (int s = 0; s < C::STAGES; ++s) mbar_init(ring.bars + s, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    // q, the cache, the metadata and the lengths may come from the preceding
+    // kernel (kv_append); the finishing kernel waits for this one
+    grid_dep_wait();
+    grid_dep_launch();
+
+    const AttendParams& a = p.at;
+    const int nf = forced_ctas(a, p.sc.scores != nullptr, gridDim.x);
+    if ((int)blockIdx.x < nf) {
+        // this CTA's chunk of the concatenated prefix/window lists
+        auto len_of = [&](int b) { return list_len(a, b); };
+        const long long total = total_units(a.batch, a.hkv, len_of);
+        const long long cpp = (total + nf - 1) / nf;
+        const long long s = (long long)blockIdx.x * cpp;
+        const long long e = min(total, s + cpp);
+        uint32_t it = 0;
+        bool ok = true;
+        attend_range<D, C::NW, C::STAGES>(a, smem, ring, it, ok, s, e, blockIdx.x);
+    } else if (p.sc.scores != nullptr) {
+        // candidate scores, tiles spread over the remaining CTAs' warps
+        uint32_t it = 0;
+        scr::score_range_bulk<D, C::STAGES>(p.sc, ring.tiles, ring.bars, it,
+                                            (blockIdx.x - nf) * C::NW + warp,
+                                            (gridDim.x - nf) * C::NW);
+    }
+}
+
+template <int D>
+cudaError_t setup_one(int* occ) {
+    cudaError_t e = cudaFuncSetAttribute(stream_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         StreamCfg<D>::SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, stream_kernel<D>,
+                                                      StreamCfg<D>::NW * 32, StreamCfg<D>::SMEM);
+    if (*occ < 1) *occ = 1;
+    return e;
+}
+
+}  // namespace
+
+cudaError_t setup_stream(DeviceCfg& d) {
+    cudaError_t e = setup_one<128>(&d.occ_stream[0]);
+    if (e == cudaSuccess) e = setup_one<256>(&d.occ_stream[1]);
+    return e;
+}
+
+int stream_chunks(int head_dim, const DeviceCfg& d) {
+    const int blocks = d.num_sms * d.occ_stream[head_dim == 128 ? 0 : 1];
+    return blocks < kMaxAttendChunks ? blocks : kMaxAttendChunks;
+}
+
+cudaError_t launch_stream(StreamParams& p, int head_dim, const DeviceCfg& d,
+                          cudaStream_t stream) {
+    const bool d128 = head_dim == 128;
+    const int blocks = stream_chunks(head_dim, d);
+    p.at.num_chunks = blocks;
+    p.at.list = kListForced;
+    if (d128)
+        return launch_pdl(stream_kernel<128>, dim3(blocks), dim3(StreamCfg<128>::NW * 32),
+                          StreamCfg<128>::SMEM, stream, 1, p);
+    return launch_pdl(stream_kernel<256>, dim3(blocks), dim3(StreamCfg<256>::NW * 32),
+                      StreamCfg<256>::SMEM, stream, 1, p);
+}
+
+}  // namespace slc

@@ -112,12 +112,38 @@ def test_decode_argument_validation():
     assert lib.slc_score_pages(FAKE, ctypes.byref(c), FAKE, 10, FAKE, 1, 8, -1, 0, FAKE,
                                None) == INVALID
     assert lib.slc_device_status(None, None) == INVALID
-    for stage in (0, 5, -1):  # only stages 1..4 exist
+    for stage in (0, 3, -1):  # only stages 1 and 2 exist
         assert lib.slc_sparse_decode_stage(stage, FAKE, ctypes.byref(c), FAKE, 10, FAKE, 1, 8, 0,
                                            0, 2, 0.0, FAKE, None, FAKE, 1 << 40,
                                            None) == INVALID
     assert lib.slc_sparse_decode_stage(2, FAKE, ctypes.byref(c), FAKE, 10, FAKE, 1, 7, 0, 0, 2,
                                        0.0, FAKE, None, FAKE, 1 << 40, None) == INVALID  # Hq % Hkv
+
+
+def test_static_entry_checks_arguments_before_size():
+    """The allocation-free entry runs the same argument checks as
+    slc_sparse_decode, before its scratch-size test."""
+    f = lib.slc_sparse_decode_static
+    f.restype = ctypes.c_int32
+    f.argtypes = [ctypes.c_void_p, ctypes.POINTER(slc._Cache), ctypes.c_void_p, ctypes.c_int32,
+                  ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                  ctypes.c_int32, ctypes.c_int32, ctypes.c_float, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p]
+    c = cache()
+
+    def call(batch=1, max_pages=10, prefix=0, window=0, budget=2, scale=0.0, q=FAKE, hq=8):
+        return f(q, ctypes.byref(c), FAKE, max_pages, FAKE, batch, hq, prefix, window, budget,
+                 scale, FAKE, None, None)
+    # shapes whose workspace would not fit the scratch array, with a bad
+    # argument: the argument error wins
+    big = dict(batch=64, max_pages=32768, budget=4096)
+    assert call(**big, prefix=-1) == INVALID
+    assert call(**big, window=-1) == INVALID
+    assert call(**big, scale=float("inf")) == INVALID
+    assert call(64, 40000, budget=4096) == UNSUPPORTED  # > 32768 candidates
+    assert call(**big, q=FAKE + 4) == INVALID
+    assert call(**big) == WORKSPACE  # well-formed but too large
+    assert call(batch=0) == OK
 
 
 def test_binding_rejects_cpu_tensors():

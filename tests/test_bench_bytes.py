@@ -23,16 +23,16 @@ def _count(x, prefix, window, budget):
     _, sel, nsel = oracle.sparse_decode(x.q, x.k_cache, x.v_cache, x.block_table, x.seq_lens,
                                         prefix, window, budget)
     hkv, D = x.k_cache.shape[1], x.k_cache.shape[3]
-    meta = kv = 0
+    meta = forced = chosen = 0
     for b, L in enumerate(x.seq_lens.tolist()):
         n, np_, ws = oracle.page_ranges(L, prefix, window)
         meta += (ws - np_) * hkv * 4 * D
         for h in range(hkv):
-            pages = set(range(np_)) | set(range(ws, n))
-            pages |= set(int(p) for p in sel[b, h, :int(nsel[b, h])])
-            tokens = sum(min(16, L - 16 * j) for j in pages)
-            kv += tokens * 4 * D
-    return meta, kv
+            fpages = set(range(np_)) | set(range(ws, n))
+            spages = set(int(p) for p in sel[b, h, :int(nsel[b, h])]) - fpages
+            forced += sum(min(16, L - 16 * j) for j in fpages) * 4 * D
+            chosen += sum(min(16, L - 16 * j) for j in spages) * 4 * D
+    return meta, forced, chosen
 
 
 def test_algorithmic_bytes_equal_what_the_oracle_reads():
@@ -40,14 +40,15 @@ def test_algorithmic_bytes_equal_what_the_oracle_reads():
                         budget=5, needles=0, seed=11, context=1000, layout="shuffled")
     x = synth.make_inputs(wl, lens_override=[1000, 333, 130])
     for prefix, window, budget in [(40, 100, 5), (0, 16, 3), (64, 256, 50), (16, 17, 0)]:
-        meta, kv = _count(x, prefix, window, budget)
+        meta, forced, chosen = _count(x, prefix, window, budget)
         total, m, k = bench.algorithmic_bytes(x.seq_lens.tolist(), 8, 2, 32, prefix, window,
                                                budget)
-        assert (m, k) == (meta, kv), (prefix, window, budget)
-        assert total == meta + kv + 3 * 8 * 32 * (2 + 4)  # q bf16 + out fp32
+        assert (m, k) == (meta, forced + chosen), (prefix, window, budget)
+        assert total == meta + forced + chosen + 3 * 8 * 32 * (2 + 4)  # q bf16 + out fp32
         st = bench.stage_bytes(x.seq_lens.tolist(), 8, 2, 32, prefix, window, budget)
-        assert st[1] == meta + 3 * 8 * 32 * 2
-        assert st[3] == kv + 3 * 8 * 32 * 2
+        assert st[1] == meta + forced + 3 * 8 * 32 * 2  # streaming kernel: + q
+        assert st[2] == chosen + 3 * 8 * 32 * (2 + 4)  # finishing kernel: + q, out
+        assert st[1] + st[2] == total + 3 * 8 * 32 * 2  # q is read by both
 
 
 def test_dense_bytes_are_every_token():

@@ -54,14 +54,18 @@ def test_build_page_meta_exact_ragged_lengths_nan_slots():
     meta_matches_oracle(Dev(x))
 
 
-def test_kv_append_matches_rebuild_and_oracle():
+@pytest.mark.parametrize("hq,hkv,D", [(8, 2, 128), (16, 2, 256), (8, 8, 256)])
+def test_kv_append_matches_rebuild_and_oracle(hq, hkv, D):
+    """Appends across page boundaries (slot 0 resets a page's bounds) at both
+    head dims: the cache holds the tokens where the host put them, and the
+    incremental bounds equal the oracle's and a rebuild, bit for bit."""
     import sparse_long_context_max_b200 as slc
-    x = small(3, 8, 2, 128, [30, 47, 16], seed=9, headroom=40)
+    x = small(3, hq, hkv, D, [30, 47, 16], seed=9 + D, headroom=40)
     d = Dev(x)
     lens = x.seq_lens.clone()
     for step in range(40):
-        kn = torch.randn((3, 2, 128), generator=torch.Generator().manual_seed(step)).to(torch.bfloat16)
-        vn = torch.randn((3, 2, 128), generator=torch.Generator().manual_seed(99 + step)).to(torch.bfloat16)
+        kn = torch.randn((3, hkv, D), generator=torch.Generator().manual_seed(step)).to(torch.bfloat16)
+        vn = torch.randn((3, hkv, D), generator=torch.Generator().manual_seed(99 + step)).to(torch.bfloat16)
         slc.kv_append(d.cache, kn.cuda(), vn.cuda(), d.bt, lens.cuda())
         for b in range(3):
             L = int(lens[b])
@@ -105,6 +109,59 @@ def test_scores_match_oracle_and_bound(tiny):
             q = x.q[0, h * G:(h + 1) * G].double()
             best = (q @ k.T).sum(0).max().item()
             assert s[0, h, j] >= best - 1e-5 * abs(best) - 1e-4
+
+
+def stream_scores(d, prefix, window, budget):
+    """The candidate scores the sparse decode itself computes (its streaming
+    kernel, stage 1), read back from the workspace: float64
+    [B][Hkv][max_pages] by page, NaN outside the candidates."""
+    import sparse_long_context_max_b200 as slc
+    x = d.x
+    B, hq, D = x.q.shape
+    hkv = x.k_cache.shape[1]
+    mp = x.block_table.shape[1]
+    ws = torch.zeros(slc.workspace_size(B, hq, hkv, D, mp, budget), dtype=torch.uint8,
+                     device="cuda")
+    slc.sparse_decode_stage(1, d.q, d.cache, d.bt, d.sl, prefix, window, budget, workspace=ws)
+    torch.cuda.synchronize()
+    assert slc.device_status() == 0
+    cs = (mp + 63) // 64 * 64  # rows by candidate, 64-float aligned
+    rows = ws[: B * hkv * cs * 4].view(torch.float32).view(B, hkv, cs).cpu().double().numpy()
+    out = np.full((B, hkv, mp), np.nan)
+    for b, L in enumerate(x.seq_lens.tolist()):
+        n, np_, wsp = oracle.page_ranges(L, prefix, window)
+        out[b, :, np_:wsp] = rows[b, :, : wsp - np_]
+    return out
+
+
+def check_scores(x, s, prefix, window, rel=2e-6):
+    """GPU scores within rel (of the largest score) of the oracle's, and never
+    below the oracle's own best group logit of a sampled page."""
+    kmin, kmax = oracle.page_bounds(x.k_cache, x.block_table, x.seq_lens)
+    so = oracle.page_scores(x.q, kmin, kmax, x.seq_lens, prefix, window)
+    cand = ~np.isnan(so)
+    assert (np.isnan(s) == ~cand).all()
+    scale = np.abs(so[cand]).max()
+    assert np.abs(s[cand] - so[cand]).max() <= rel * scale
+    return so
+
+
+def test_stream_scores_match_oracle_decode256k():
+    """The decode path's own scores at 256k (group 8, d 128): every candidate
+    of every unit within 2e-6 (relative) of the oracle."""
+    x = synth.make_inputs(W["decode256k"])
+    d = Dev(x)
+    check_scores(x, stream_scores(d, x.prefix, x.window, x.budget), x.prefix, x.window)
+
+
+def test_stream_scores_match_oracle_layers131k():
+    """The same at d 256 (one layer of the 131k plan, group 8)."""
+    wl = W["layers131k"]
+    plan = synth.layer_plan(wl)
+    layer = [i for i, (_, _, dn) in enumerate(plan) if not dn][0]
+    x = synth.make_inputs(wl, layer=layer)
+    d = Dev(x)
+    check_scores(x, stream_scores(d, x.prefix, x.window, x.budget), x.prefix, x.window)
 
 
 def test_select_exact_on_given_scores():
@@ -159,9 +216,55 @@ def test_sparse_attend_with_another_layers_selection():
     check_output(y, out.cpu().double().numpy(), x.prefix, x.window, sel)
 
 
+def test_sparse_attend_union_semantics():
+    """A given selection is attended as a set united with the prefix and
+    window: entries that are prefix or window pages add nothing, -1 is
+    padding, and out-of-range or out-of-order entries are skipped and
+    flagged.  Compared with the oracle, whose attended set is that union."""
+    import sparse_long_context_max_b200 as slc
+    x = small(2, 8, 2, 128, [3000, 1000], prefix=32, window=128, budget=8, seed=31)
+    d = Dev(x)
+    n0, np0, ws0 = oracle.page_ranges(3000, 32, 128)
+    n1, np1, ws1 = oracle.page_ranges(1000, 32, 128)
+    sel = np.full((2, 2, 8), -1, dtype=np.int32)
+    sel[0, 0, :6] = [0, 5, 40, 100, ws0, n0 - 1]  # prefix, candidates, window pages
+    sel[0, 1, :3] = [7, 9, 11]
+    sel[1, 0, :4] = [3, 4, ws1 + 1, n1 - 1]
+    sel[1, 1, :2] = [np1, ws1 - 1]
+    out = slc.sparse_attend(d.q, d.cache, d.bt, d.sl, 32, 128, torch.from_numpy(sel).cuda())
+    torch.cuda.synchronize()
+    assert slc.device_status() == 0
+    check_output(x, out.cpu().double().numpy(), 32, 128, sel)
+    bad = sel.copy()
+    bad[0, 0, 6] = n0 + 5  # past the sequence
+    bad[1, 1, 2] = 1  # not above the entry before it
+    out2 = slc.sparse_attend(d.q, d.cache, d.bt, d.sl, 32, 128, torch.from_numpy(bad).cuda())
+    torch.cuda.synchronize()
+    assert slc.device_status() & 4  # bad selection, skipped
+    check_output(x, out2.cpu().double().numpy(), 32, 128, sel)
+
+
+@pytest.mark.parametrize("lens,budget", [([5000, 9000, 700], 37), ([262144 // 8, 3000], 300)])
+def test_selection_ties_go_to_the_lower_page(lens, budget):
+    """Keys of +-1 only: nearly every page has the bounds (-1, +1) in every
+    dimension, so nearly every candidate has the same score, computed the
+    same way on the GPU.  The selection must then be the lowest-indexed of
+    the top-scoring pages, exactly: the tie-break of the method's total
+    order, exercised across all CTAs of a cluster."""
+    x = small(len(lens), 8, 2, 128, lens, prefix=64, window=256, budget=budget, seed=41)
+    x.k_cache = torch.where(x.k_cache >= 0, 1.0, -1.0).to(torch.bfloat16)
+    d = Dev(x)
+    out, sel = d.sparse()
+    kmin, kmax = oracle.page_bounds(x.k_cache, x.block_table, x.seq_lens)
+    so = oracle.page_scores(x.q, kmin, kmax, x.seq_lens, x.prefix, x.window)
+    want, _ = oracle.select_pages(so, x.seq_lens, x.prefix, x.window, budget)
+    np.testing.assert_array_equal(sel, want)
+    check_output(x, out, x.prefix, x.window, sel)
+
+
 def test_stages_in_order_equal_one_call():
-    """slc_sparse_decode_stage 1..4 on one workspace reproduce slc_sparse_decode
-    bit for bit (same kernels, same order)."""
+    """slc_sparse_decode_stage 1 then 2 on one workspace reproduce
+    slc_sparse_decode bit for bit (same kernels, same order)."""
     import sparse_long_context_max_b200 as slc
     x = synth.make_inputs(W["ragged"])
     d = Dev(x)
@@ -175,14 +278,14 @@ def test_stages_in_order_equal_one_call():
                              selected_out=sel1, workspace=ws)
     out2 = torch.full_like(out1, float("nan"))
     ws.zero_()
-    for stage in (1, 2, 3, 4):
+    for stage in (1, 2):
         slc.sparse_decode_stage(stage, d.q, d.cache, d.bt, d.sl, x.prefix, x.window, x.budget,
                                 out=out2, selected_out=sel2, workspace=ws)
     torch.cuda.synchronize()
     assert slc.device_status() == 0
     assert torch.equal(sel1, sel2)
     assert torch.equal(out1, out2)
-    for bad in (0, 5, -1):
+    for bad in (0, 3, -1):
         with pytest.raises(slc.SLCError):
             slc.sparse_decode_stage(bad, d.q, d.cache, d.bt, d.sl, x.prefix, x.window, x.budget,
                                     out=out2, selected_out=sel2, workspace=ws)
