@@ -57,6 +57,12 @@ def _load(path=None):
             lib.oracle_sparse_decode.argtypes = [P, P, P, I, I, I, I, P, I, P, I,
                                                  I, I, I, ctypes.c_double, P, P, P]
             lib.oracle_sparse_decode.restype = I
+            lib.oracle_fp8_value.argtypes = [I]
+            lib.oracle_fp8_value.restype = ctypes.c_double
+            lib.oracle_fp8_round.argtypes = [ctypes.c_double, I]
+            lib.oracle_fp8_round.restype = I
+            lib.oracle_page_bounds_fp8.argtypes = [P, I, I, I, P, I, P, I, P, P]
+            lib.oracle_page_bounds_fp8.restype = I
             if path is not None:
                 return lib
             _lib = lib
@@ -126,6 +132,42 @@ def page_bounds(k_cache, block_table, seq_lens):
     kmax = np.full((B, hkv, max_pages, dim), np.nan)
     rc = lib.oracle_page_bounds(_ptr(k), num_pages, hkv, dim, _ptr(bt), max_pages,
                                 _ptr(sl), B, _ptr(kmin), _ptr(kmax))
+    if rc:
+        raise ValueError("block table entry outside the page pool")
+    return kmin, kmax
+
+
+def fp8_value(code: int) -> float:
+    """Value of an E4M3 code (NaN codes: +-the largest bf16, the
+    out-of-range bound of their sign)."""
+    return _load().oracle_fp8_value(int(code))
+
+
+def fp8_round(x: float, up: bool) -> int:
+    """Outward rounding to E4M3: up -> smallest value >= x, else largest
+    value <= x (0x7F / 0xFF beyond the range)."""
+    return _load().oracle_fp8_round(float(x), int(bool(up)))
+
+
+def fp8_decode(codes) -> np.ndarray:
+    """E4M3 codes (any shape, uint8) -> float64 values."""
+    table = np.array([fp8_value(c) for c in range(256)])
+    return table[np.asarray(codes, dtype=np.uint8)]
+
+
+def page_bounds_fp8(k_cache, block_table, seq_lens):
+    """E4M3 page bounds, rounded outward: two uint8 code arrays
+    [B][Hkv][max_pages][D] (kmin rounded down, kmax up); pages past the
+    sequence are 0."""
+    lib = _load()
+    k = _bits(k_cache)
+    bt, sl = _i32(block_table), _i32(seq_lens)
+    num_pages, hkv, page, dim = k.shape
+    B, max_pages = bt.shape
+    kmin = np.zeros((B, hkv, max_pages, dim), dtype=np.uint8)
+    kmax = np.zeros((B, hkv, max_pages, dim), dtype=np.uint8)
+    rc = lib.oracle_page_bounds_fp8(_ptr(k), num_pages, hkv, dim, _ptr(bt), max_pages,
+                                    _ptr(sl), B, _ptr(kmin), _ptr(kmax))
     if rc:
         raise ValueError("block table entry outside the page pool")
     return kmin, kmax

@@ -123,6 +123,119 @@ int oracle_page_bounds(const uint16_t *k_cache, int num_pages, int hkv, int dim,
     return 0;
 }
 
+/* Low-precision page metadata (the bounds stored in 8 bits, a quarter of
+ * the bytes the scoring reads at head_dim 128; cf. "Faster Than Flash: Fudan
+ * FFD Hits 11.6x Kernel Speedup, Pushes Long-Context Decoding to 256K",
+ * section "The Hard Constraint on an Old Problem": a low-bit scan of the
+ * blocks).  Format: 8-bit floating point E4M3 ("FN" form: 1 sign bit, 4
+ * exponent bits with bias 7, 3 mantissa bits; exponent field 0 is
+ * subnormal; no infinities; 0x7F / 0xFF are NaN).  To keep the score an
+ * upper bound the bounds round OUTWARD: kmin to the largest E4M3 value <=
+ * kmin, kmax to the smallest E4M3 value >= kmax.  A bound beyond the format's
+ * range (|x| > 448) is stored as the NaN code of its sign and read back as
+ * the largest bf16 value of that sign (so it still bounds any bf16 key).
+ * Zero is always code 0x00. */
+
+#define BF16_MAX 3.3895313892515355e38 /* 0x7F7F */
+
+/* The value of an E4M3 code, from the format definition (NaN codes: the
+ * out-of-range bound of their sign, +-BF16_MAX). */
+double oracle_fp8_value(int code)
+{
+    int sgn = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7)
+        v = BF16_MAX;
+    else if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+typedef struct {
+    double v;
+    int code;
+} fp8_entry_t;
+
+static fp8_entry_t fp8_table[256];
+static int fp8_count = 0;
+
+static int fp8_cmp(const void *x, const void *y)
+{
+    double a = ((const fp8_entry_t *)x)->v, b = ((const fp8_entry_t *)y)->v;
+    return (a > b) - (a < b);
+}
+
+/* Every finite E4M3 value once, ascending (-0 left out: zero is 0x00). */
+static void fp8_build_table(void)
+{
+    if (fp8_count)
+        return;
+    int n = 0;
+    for (int c = 0; c < 256; c++) {
+        if ((c & 0x7F) == 0x7F || c == 0x80)
+            continue;
+        fp8_table[n].v = oracle_fp8_value(c);
+        fp8_table[n].code = c;
+        n++;
+    }
+    qsort(fp8_table, n, sizeof(fp8_entry_t), fp8_cmp);
+    fp8_count = n;
+}
+
+/* Outward rounding of x to E4M3: up != 0 gives the smallest value >= x
+ * (0x7F if x > 448), else the largest value <= x (0xFF if x < -448). */
+int oracle_fp8_round(double x, int up)
+{
+    fp8_build_table();
+    /* binary search: first entry with value >= x */
+    int lo = 0, hi = fp8_count;
+    while (lo < hi) {
+        int mid = (lo + hi) / 2;
+        if (fp8_table[mid].v < x)
+            lo = mid + 1;
+        else
+            hi = mid;
+    }
+    if (up)
+        return lo < fp8_count ? fp8_table[lo].code : 0x7F;
+    if (lo < fp8_count && fp8_table[lo].v == x)
+        return fp8_table[lo].code;
+    return lo > 0 ? fp8_table[lo - 1].code : 0xFF;
+}
+
+/* Step: E4M3 page bounds.  The exact bounds of oracle_page_bounds, each
+ * rounded outward: kmin down, kmax up.  Codes [B][Hkv][max_pages][D] for
+ * pages j < n_b (others left as they are).  Returns 0, or -1 on a
+ * block-table entry outside the pool. */
+int oracle_page_bounds_fp8(const uint16_t *k_cache, int num_pages, int hkv, int dim,
+                           const int32_t *block_table, int max_pages,
+                           const int32_t *seq_lens, int batch, uint8_t *kmin8,
+                           uint8_t *kmax8)
+{
+    int64_t nb = (int64_t)batch * hkv * max_pages * dim;
+    double *kmin = (double *)malloc(sizeof(double) * (nb > 0 ? nb : 1));
+    double *kmax = (double *)malloc(sizeof(double) * (nb > 0 ? nb : 1));
+    int rc = oracle_page_bounds(k_cache, num_pages, hkv, dim, block_table, max_pages,
+                                seq_lens, batch, kmin, kmax);
+    for (int b = 0; b < batch && rc == 0; b++) {
+        int L = seq_lens[b];
+        int n = L > 0 ? (L + PAGE - 1) / PAGE : 0;
+        for (int h = 0; h < hkv; h++)
+            for (int j = 0; j < n; j++) {
+                int64_t base = (((int64_t)b * hkv + h) * max_pages + j) * dim;
+                for (int d = 0; d < dim; d++) {
+                    kmin8[base + d] = (uint8_t)oracle_fp8_round(kmin[base + d], 0);
+                    kmax8[base + d] = (uint8_t)oracle_fp8_round(kmax[base + d], 1);
+                }
+            }
+    }
+    free(kmin);
+    free(kmax);
+    return rc;
+}
+
 /* Step: score every candidate page with the Quest bound, summed over the
  * query heads that share the kv head.  Written literally, one max per
  * (query head, dimension).  Output [B][Hkv][max_pages]; non-candidate

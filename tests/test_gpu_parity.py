@@ -456,3 +456,70 @@ def test_layers131k_sampled_layers():
             check_output(x, out, x.prefix, x.window, sel)
         del d, x
         torch.cuda.empty_cache()
+
+
+def test_layers131k_graph_step_all_layers():
+    """One decode step of the 15-layer plan at 131072 tokens (d 256), replayed
+    from its CUDA graph: per layer the new token's append, then the layer's
+    decode.  Cross-layer reuse is on ("IndexCache: cross-layer reuse speeds
+    30B prefill 1.82x": Full layers select, Shared layers attend the nearest
+    Full layer's selection with their own window).  Checked per layer: the
+    appended token landed, Full layers' selections against the oracle's
+    (tie band), every sparse layer's output against the oracle attending
+    prefix + window + the selection it used, the dense layers on a sampled
+    sequence."""
+    import sparse_long_context_max_b200 as slc
+    from sparse_long_context_max_b200 import plan as P
+    wl = W["layers131k"]
+    x = synth.make_inputs(wl, layer=0, headroom_tokens=16)
+    layers = synth.layer_plan(wl)
+    specs = P.index_reuse([P.LayerSpec(w, k, dn) for w, k, dn in layers])
+    assert any(s.shared for s in specs) and any(s.dense for s in specs)
+    k0, v0 = x.k_cache.cuda(), x.v_cache.cuda()
+    bt = x.block_table.cuda()
+    caches = []
+    for _ in specs:
+        c = slc.PagedCache(k0.clone(), v0.clone())
+        slc.build_page_meta(c, bt, x.seq_lens.cuda())
+        caches.append(c)
+    del k0, v0
+    step = P.DecodeStep(caches, bt, specs, wl.prefix, wl.hq)
+    toks = [synth.step_tokens(wl, 1, layer=i) for i in range(len(specs))]
+    for i, (q, kn, vn) in enumerate(toks):
+        step.q[i].copy_(q)
+        step.k_new[i].copy_(kn)
+        step.v_new[i].copy_(vn)
+    step.positions.copy_(x.seq_lens)
+    step.seq_lens.copy_(x.seq_lens + 1)
+    step.capture()
+    step.replay()  # the append writes the same slot again: idempotent
+    torch.cuda.synchronize()
+    assert slc.device_status() == 0
+    lens1 = x.seq_lens + 1
+    for i, s in enumerate(specs):
+        q, kn, vn = toks[i]
+        y = slice_batch(x, list(range(wl.batch)))
+        y.q, y.seq_lens = q, lens1
+        y.k_cache, y.v_cache = x.k_cache.clone(), x.v_cache.clone()
+        for b in range(wl.batch):
+            L = int(x.seq_lens[b])
+            phys = int(x.block_table[b, L // 16])
+            y.k_cache[phys, :, L % 16] = kn[b]
+            y.v_cache[phys, :, L % 16] = vn[b]
+        got = caches[i]
+        for b in range(wl.batch):
+            L = int(x.seq_lens[b])
+            phys = int(x.block_table[b, L // 16])
+            assert torch.equal(got.k_cache[phys, :, L % 16].cpu(), kn[b])
+        out = step.out[i].cpu().double().numpy()
+        if s.dense:
+            check_output(slice_batch(y, [3]), out[[3]], 0, 0, None, dense=True)
+            continue
+        if not s.shared:
+            sel = step.selected[i].cpu().numpy()
+            check_selection(y, sel, wl.prefix, s.window, s.budget)
+        else:
+            sel = step.selected[step.full_of[i]].cpu().numpy()
+        check_output(y, out, wl.prefix, s.window, sel)
+    del caches, step
+    torch.cuda.empty_cache()

@@ -328,3 +328,95 @@ def test_needles_are_selected_tiny_workload():
         chosen = set(sel[0, h].tolist())
         for t in x.needle_tokens[0]:
             assert t // 16 in chosen
+
+
+# ---------------------------------------------------------------- fp8 metadata
+
+def test_fp8_rounding_golden():
+    """Hand-worked E4M3 outward roundings (tests/golden/fp8_rounding.json)."""
+    for c in _load("fp8_rounding.json")["cases"]:
+        assert oracle.fp8_round(c["x"], True) == c["up"], c
+        assert oracle.fp8_round(c["x"], False) == c["down"], c
+
+
+def _e4m3_table():
+    """Every finite E4M3 value, from torch's float8_e4m3fn dtype (a library
+    definition of the format, independent of the oracle)."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    vals = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    return codes.numpy(), vals
+
+
+def test_fp8_values_match_library_format():
+    codes, vals = _e4m3_table()
+    for c, v in zip(codes, vals):
+        if np.isnan(v):  # the two NaN codes: the out-of-range bounds
+            assert abs(oracle.fp8_value(int(c))) == 3.3895313892515355e38
+            assert (oracle.fp8_value(int(c)) > 0) == (c == 0x7F)
+        else:
+            assert oracle.fp8_value(int(c)) == v, c
+
+
+def test_fp8_rounding_is_outward_and_tight():
+    """For bf16 values over the whole range (tiny, subnormal in E4M3, normal,
+    beyond 448): down <= x <= up, and no E4M3 value lies strictly between x
+    and either (checked against the library's value table)."""
+    _, vals = _e4m3_table()
+    finite = np.unique(vals[~np.isnan(vals)])
+    g = torch.Generator().manual_seed(7)
+    xs = torch.cat([torch.randn(3000, generator=g) * s for s in (1e-3, 0.05, 1.0, 30.0, 600.0)])
+    xs = xs.to(torch.bfloat16).double().numpy()
+    for x in xs:
+        up, dn = oracle.fp8_round(x, True), oracle.fp8_round(x, False)
+        vu, vd = oracle.fp8_value(up), oracle.fp8_value(dn)
+        assert vd <= x <= vu, (x, vd, vu)
+        assert not ((finite > x) & (finite < vu)).any(), x
+        assert not ((finite < x) & (finite > vd)).any(), x
+
+
+def test_fp8_page_bounds_round_the_exact_bounds_outward():
+    """E4M3 page bounds are the exact bounds rounded outward, and the score
+    from them bounds the score from the exact bounds, which bounds every
+    group logit of the page (fp64)."""
+    x = _small_cache(2, 8, 2, 64, [400, 333], seed=13)
+    x.k_cache = (x.k_cache.float() * 3).to(torch.bfloat16)  # some keys beyond +-1
+    kmin, kmax = oracle.page_bounds(x.k_cache, x.block_table, x.seq_lens)
+    c8min, c8max = oracle.page_bounds_fp8(x.k_cache, x.block_table, x.seq_lens)
+    m8, M8 = oracle.fp8_decode(c8min), oracle.fp8_decode(c8max)
+    for b, L in enumerate(x.seq_lens.tolist()):
+        n = -(-L // 16)
+        assert (m8[b, :, :n] <= kmin[b, :, :n]).all()
+        assert (M8[b, :, :n] >= kmax[b, :, :n]).all()
+        for h in range(2):
+            for j in range(n):
+                for d in range(0, 64, 7):
+                    assert c8min[b, h, j, d] == oracle.fp8_round(kmin[b, h, j, d], False)
+                    assert c8max[b, h, j, d] == oracle.fp8_round(kmax[b, h, j, d], True)
+    s = oracle.page_scores(x.q, kmin, kmax, x.seq_lens, prefix=16, window=48)
+    s8 = oracle.page_scores(x.q, m8, M8, x.seq_lens, prefix=16, window=48)
+    cand = ~np.isnan(s)
+    assert (s8[cand] >= s[cand]).all()
+    for b in range(2):
+        for h in range(2):
+            for j in np.nonzero(cand[b, h])[0][::5]:
+                assert s8[b, h, j] >= _group_dots(x, b, h, j).sum(axis=0).max() - 1e-9
+
+
+def test_fp8_bounds_of_a_page_grow_one_token_at_a_time():
+    """Outward rounding is monotone, so the bounds of a page with one more
+    token are the old codes combined with the new token's rounded values
+    (min of the downs, max of the ups): appending keeps fp8 metadata exact."""
+    x = _small_cache(1, 4, 2, 32, [16], seed=17)
+    bt = x.block_table
+    for t in range(1, 16):
+        a8 = oracle.page_bounds_fp8(x.k_cache, bt, [t])
+        b8 = oracle.page_bounds_fp8(x.k_cache, bt, [t + 1])
+        k = x.k_cache[int(bt[0, 0]), :, t].double().numpy()  # [Hkv][D]
+        for h in range(2):
+            for d in range(32):
+                dn = oracle.fp8_round(k[h, d], False)
+                up = oracle.fp8_round(k[h, d], True)
+                lo = min(oracle.fp8_value(a8[0][0, h, 0, d]), oracle.fp8_value(dn))
+                hi = max(oracle.fp8_value(a8[1][0, h, 0, d]), oracle.fp8_value(up))
+                assert oracle.fp8_value(b8[0][0, h, 0, d]) == lo
+                assert oracle.fp8_value(b8[1][0, h, 0, d]) == hi

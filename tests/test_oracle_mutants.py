@@ -38,6 +38,11 @@ MUTANTS = [
      "int k = budget < m ? budget + 1 : m;"),
     ("sparse drops window pages", "for (int j = ws; j < n; j++)\n                    use[j] = 1;",
      "for (int j = ws + 1; j < n; j++)\n                    use[j] = 1;"),
+    ("fp8 bounds round to nearest",
+     "kmax8[base + d] = (uint8_t)oracle_fp8_round(kmax[base + d], 1);",
+     "kmax8[base + d] = (uint8_t)oracle_fp8_round(kmax[base + d], kmax[base + d] - oracle_fp8_value(oracle_fp8_round(kmax[base + d], 0)) > oracle_fp8_value(oracle_fp8_round(kmax[base + d], 1)) - kmax[base + d]);"),
+    ("fp8 rounding off by one code", "return lo < fp8_count ? fp8_table[lo].code : 0x7F;",
+     "return lo + 1 < fp8_count ? fp8_table[lo + 1].code : 0x7F;"),
 ]
 
 
