@@ -36,7 +36,8 @@
  *
  * Layouts (row-major, innermost last):
  *   K, V cache   bf16 [num_pages][num_kv_heads][16][head_dim]
- *   page meta    bf16 [num_pages][num_kv_heads][2][head_dim]  (kmin, kmax)
+ *   page meta    [num_pages][num_kv_heads][2][head_dim] (kmin, kmax): bf16,
+ *                or 8-bit E4M3 rounded outward (slc_cache_t.meta_format)
  *   q            bf16 [batch][num_q_heads][head_dim]
  *   block_table  int32 [batch][max_pages_per_seq]: logical page -> physical
  *   seq_lens     int32 [batch]: tokens in each sequence (the decode query's
@@ -92,8 +93,26 @@ enum {
     SLC_STATUS_WAIT_TIMEOUT = 8   /* a bounded wait on a bulk copy gave up */
 };
 
+/* Page metadata formats (slc_cache_t.meta_format). */
+enum {
+    /* bf16 [num_pages][num_kv_heads][2][head_dim]: kmin, kmax exactly */
+    SLC_META_BF16 = 0,
+    /* uint8 [num_pages][num_kv_heads][2][head_dim]: kmin and kmax as 8-bit
+     * floats E4M3 (OCP "FN": bias 7, 3 mantissa bits, no infinities),
+     * rounded OUTWARD -- kmin to the largest E4M3 value <= kmin, kmax to the
+     * smallest >= kmax -- so the score stays an upper bound of q.k over the
+     * page.  A bound beyond +-448 is stored as the NaN code of its sign
+     * (0x7F / 0xFF) and read as the largest bf16 value of that sign; zero is
+     * 0x00.  Half the metadata bytes the scoring reads.  (Low-bit scanning:
+     * "Faster Than Flash: Fudan FFD Hits 11.6x Kernel Speedup, Pushes
+     * Long-Context Decoding to 256K", section "The Hard Constraint on an Old
+     * Problem".) */
+    SLC_META_FP8_E4M3 = 1
+};
+
 /* The paged cache of one layer.  head_dim must be 128 or 256, page_size 16.
- * num_q_heads / num_kv_heads (the GQA group) must be 1..8. */
+ * num_q_heads / num_kv_heads (the GQA group) must be 1..8.  meta_format is
+ * one of SLC_META_*; the metadata buffer has the layout of that format. */
 typedef struct slc_cache {
     void *k_cache;
     void *v_cache;
@@ -102,6 +121,7 @@ typedef struct slc_cache {
     int32_t num_kv_heads;
     int32_t head_dim;
     int32_t page_size;
+    int32_t meta_format;
 } slc_cache_t;
 
 /* Append one decode token per sequence.  Writes k_new[b][h] / v_new[b][h]

@@ -26,7 +26,7 @@ __all__ = [
     "SLCError", "PagedCache", "kv_append", "build_page_meta", "workspace_size",
     "score_pages", "select_pages", "sparse_decode", "sparse_attend", "dense_decode",
     "device_status",
-    "library_path", "KERNELS_PER_CALL", "STATUS_BITS",
+    "library_path", "KERNELS_PER_CALL", "STATUS_BITS", "META_FORMATS",
 ]
 
 PAGE = 16
@@ -50,7 +50,11 @@ class _Cache(ctypes.Structure):
     _fields_ = [("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
                 ("meta", ctypes.c_void_p), ("num_pages", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("page_size", ctypes.c_int32)]
+                ("page_size", ctypes.c_int32), ("meta_format", ctypes.c_int32)]
+
+
+# page metadata formats (include/slc.h SLC_META_*)
+META_FORMATS = {"bf16": 0, "fp8": 1}
 
 
 def _load() -> ctypes.CDLL:
@@ -119,23 +123,32 @@ def _need(t, dtype, name, ndim=None):
 
 
 class PagedCache:
-    """One layer's paged K/V cache plus its page metadata (device tensors)."""
+    """One layer's paged K/V cache plus its page metadata (device tensors).
+
+    meta_format "bf16" keeps each page's key min/max exactly (bf16
+    [num_pages][Hkv][2][D]); "fp8" keeps them as 8-bit E4M3 rounded outward
+    (uint8, same shape: half the bytes the scoring reads)."""
 
     def __init__(self, k_cache: torch.Tensor, v_cache: torch.Tensor,
-                 meta: torch.Tensor | None = None):
+                 meta: torch.Tensor | None = None, meta_format: str = "bf16"):
         _need(k_cache, torch.bfloat16, "k_cache", 4)
         _need(v_cache, torch.bfloat16, "v_cache", 4)
         if k_cache.shape != v_cache.shape or k_cache.shape[2] != PAGE:
             raise ValueError("k/v cache must be [num_pages][Hkv][16][D] and equal")
+        if meta_format not in META_FORMATS:
+            raise ValueError("meta_format must be one of %s" % sorted(META_FORMATS))
         n, hkv, _, d = k_cache.shape
+        mdt = torch.bfloat16 if meta_format == "bf16" else torch.uint8
         if meta is None:
-            meta = torch.empty((n, hkv, 2, d), dtype=torch.bfloat16, device=k_cache.device)
-        _need(meta, torch.bfloat16, "meta", 4)
+            meta = torch.empty((n, hkv, 2, d), dtype=mdt, device=k_cache.device)
+        _need(meta, mdt, "meta", 4)
         if tuple(meta.shape) != (n, hkv, 2, d):
             raise ValueError("meta must be [num_pages][Hkv][2][D]")
         self.k_cache, self.v_cache, self.meta = k_cache, v_cache, meta
+        self.meta_format = meta_format
         self.num_pages, self.num_kv_heads, self.head_dim = n, hkv, d
-        self._c = _Cache(k_cache.data_ptr(), v_cache.data_ptr(), meta.data_ptr(), n, hkv, d, PAGE)
+        self._c = _Cache(k_cache.data_ptr(), v_cache.data_ptr(), meta.data_ptr(), n, hkv, d, PAGE,
+                         META_FORMATS[meta_format])
 
     @property
     def c(self):

@@ -72,6 +72,8 @@ int check_cache(const slc_cache_t* c) {
     if (c->page_size != kPage) return SLC_ERR_UNSUPPORTED;
     if (c->head_dim != 128 && c->head_dim != 256) return SLC_ERR_UNSUPPORTED;
     if (c->num_kv_heads <= 0 || c->num_pages <= 0) return SLC_ERR_INVALID_ARG;
+    if (c->meta_format != SLC_META_BF16 && c->meta_format != SLC_META_FP8_E4M3)
+        return SLC_ERR_UNSUPPORTED;
     if (!c->k_cache || !c->v_cache || !c->meta) return SLC_ERR_INVALID_ARG;
     if (!aligned16(c->k_cache) || !aligned16(c->v_cache) || !aligned16(c->meta))
         return SLC_ERR_INVALID_ARG;
@@ -154,7 +156,8 @@ int slc_kv_append(const slc_cache_t* cache, const void* k_new, const void* v_new
     if ((rc = device_cfg(&dev))) return rc;
     KvAppendParams p{k_new,     v_new,     cache->k_cache,          cache->v_cache,
                      cache->meta, block_table, positions,            dev->status,
-                     batch,     cache->num_kv_heads, max_pages_per_seq, cache->num_pages};
+                     batch,     cache->num_kv_heads, max_pages_per_seq, cache->num_pages,
+                     cache->meta_format};
     cudaError_t e = launch_kv_append(p, cache->head_dim, stream);
     return e == cudaSuccess ? SLC_OK : note_cuda(e);
 }
@@ -170,7 +173,8 @@ int slc_build_page_meta(const slc_cache_t* cache, const int32_t* block_table,
     const DeviceCfg* dev;
     if ((rc = device_cfg(&dev))) return rc;
     BuildMetaParams p{cache->k_cache, cache->meta, block_table, seq_lens, dev->status, batch,
-                      cache->num_kv_heads, max_pages_per_seq, cache->num_pages};
+                      cache->num_kv_heads, max_pages_per_seq, cache->num_pages,
+                      cache->meta_format};
     cudaError_t e = launch_build_meta(p, cache->head_dim, *dev, stream);
     return e == cudaSuccess ? SLC_OK : note_cuda(e);
 }
@@ -191,7 +195,8 @@ int slc_score_pages(const void* q, const slc_cache_t* cache, const int32_t* bloc
     ScoreParams p{q,           cache->meta, block_table, seq_lens,
                   scores,      dev->status, batch,
                   num_q_heads, cache->num_kv_heads, num_q_heads / cache->num_kv_heads,
-                  max_pages_per_seq, cache->num_pages, prefix, window, 0, nullptr};
+                  max_pages_per_seq, cache->num_pages, prefix, window, 0, nullptr,
+                  cache->meta_format};
     cudaError_t e = launch_score(p, cache->head_dim, *dev, stream);
     return e == cudaSuccess ? SLC_OK : note_cuda(e);
 }
@@ -297,7 +302,7 @@ static int decode(int mode, const void* q, const slc_cache_t* cache,
     sp.sc = ScoreParams{q,           cache->meta, block_table, seq_lens,
                         scoring ? scores : nullptr, dev->status, batch,
                         num_q_heads, hkv,         num_q_heads / hkv, max_pages_per_seq,
-                        cache->num_pages, prefix, window, cs, tile_max};
+                        cache->num_pages, prefix, window, cs, tile_max, cache->meta_format};
     if (stage == 0 || stage == 1) {
         e = launch_stream(sp, D, *dev, stream);
         if (e != cudaSuccess) return note_cuda(e, "stream");

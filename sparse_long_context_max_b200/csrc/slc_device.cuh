@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -47,6 +48,65 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     if (f == 0.f) f = 0.f;  // -0 and +0 tie
     const uint32_t u = __float_as_uint(f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// ---------------------------------------------------------------- E4M3
+// 8-bit floats E4M3 (OCP "FN": sign, 4 exponent bits with bias 7, 3
+// mantissa bits; exponent field 0 is subnormal, m/8 * 2^-6; no infinities;
+// 0x7F / 0xFF are NaN; the largest finite value is 448).  Page bounds are
+// rounded outward and a bound beyond the range keeps the NaN code of its
+// sign, read back as the largest bf16 of that sign.
+
+constexpr float kBf16Max = 3.38953139e38f;  // bf16 0x7F7F
+
+// x rounded to E4M3: up -> the smallest value >= x, else the largest value
+// <= x; beyond +-448 the NaN code of the rounding's side; zero (and a NaN
+// key, conservatively out of range) as documented above.
+__device__ __forceinline__ uint32_t e4m3_round(float x, bool up) {
+    if (x != x) return up ? 0x7Fu : 0xFFu;
+    if (x == 0.f) return 0u;
+    const bool neg = x < 0.f;
+    const float a = fabsf(x);
+    const bool away = up != neg;  // round the magnitude away from zero?
+    if (a > 448.f) return away ? (neg ? 0xFFu : 0x7Fu) : (neg ? 0xFEu : 0x7Eu);
+    int e = (int)((__float_as_uint(a) >> 23) & 0xFF) - 127;  // floor(log2 a)
+    if (e < -6) e = -6;  // below the normal range the grid step stays 2^-9
+    // the magnitude in units of the grid step 2^(e-3): exact (power of two)
+    const float q = ldexpf(a, 3 - e);
+    int mi = (int)(away ? ceilf(q) : floorf(q));  // 0 .. 16
+    if (mi == 0) return 0u;
+    if (mi == 16) {  // carried into the next binade
+        ++e;
+        mi = 8;
+    }
+    const uint32_t E = mi < 8 ? 0u : (uint32_t)(e + 7);  // mi < 8 only for subnormals
+    const uint32_t M = mi < 8 ? (uint32_t)mi : (uint32_t)(mi - 8);
+    return (neg ? 0x80u : 0u) | (E << 3) | M;
+}
+
+// The value of an E4M3 code (NaN codes: +-kBf16Max).
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+    const uint32_t E = (c >> 3) & 15u, M = c & 7u;
+    float v;
+    if (E == 15u && M == 7u)
+        v = kBf16Max;
+    else if (E == 0u)
+        v = ldexpf((float)M, -9);
+    else
+        v = ldexpf((float)(8u + M), (int)E - 10);
+    return (c & 0x80u) ? -v : v;
+}
+
+// Two E4M3 codes (low byte first) -> two floats, the NaN codes read as
+// `oor` (+-kBf16Max: the out-of-range bound of the row).
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two, float oor) {
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((unsigned short)two));
+    const __half2 hv = *reinterpret_cast<const __half2*>(&h);
+    float2 f = __half22float2(hv);
+    f.x = f.x == f.x ? f.x : oor;
+    f.y = f.y == f.y ? f.y : oor;
+    return f;
 }
 
 // ---------------------------------------------------------------- bf16
@@ -178,12 +238,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         : "memory");
 }
 
-// 16-byte asynchronous global -> shared copy (LSU path), grouped per thread.
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
-                 : "memory");
-}
-
 // 4-byte asynchronous global -> shared copy (both 4-byte aligned).
 __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src)
@@ -211,6 +265,12 @@ __device__ __forceinline__ void grid_dep_launch() {
 // Hint: bring `bytes` (a multiple of 16) at p (16-byte aligned) into L2.
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ uint2 lds64(const void* p) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_addr(p)));
+    return v;
 }
 
 __device__ __forceinline__ uint4 lds128(const void* p) {

@@ -46,17 +46,16 @@ namespace {
 namespace cg = cooperative_groups;
 using namespace attn;
 
-// Two CTAs must fit on an SM so that one cluster per unit is co-resident for
-// the usual unit counts.  At d = 128: eight warps of at most 128 registers,
-// all attending with one ring stage each (two warps per scheduler hide each
-// other's latencies); at d = 256 the attention needs ~250 registers, so four
-// warps.
+// Four warps, all attending: the attention needs ~150 (d = 128) to ~250
+// (d = 256) registers per thread, and two CTAs must fit on an SM so that one
+// cluster per unit is co-resident for the usual unit counts.  (Eight warps
+// of 128 registers with one ring stage each measured slower.)
 template <int D>
 struct FinishCfg {
-    static constexpr int NT = D == 128 ? 256 : 128;    // threads per CTA
+    static constexpr int NT = 128;                     // threads per CTA
     static constexpr int NW = NT / 32;                 // warps per CTA
     static constexpr int NW_ATT = NW;                  // warps that attend
-    static constexpr int STAGES = 1;                   // ring stages per attending warp
+    static constexpr int STAGES = D == 128 ? 2 : 1;    // ring stages per attending warp
     static constexpr int RING = STAGES * 2 * kPage * D * 2;
     static constexpr int MIN_BLOCKS = 2;
 };
@@ -274,18 +273,19 @@ __device__ void cluster_kth(cg::cluster_group& cl, const uint32_t* keys, int cnt
     }
 }
 
-// The k-th largest of n keys held by this CTA (key_at(i), i < n), by the
+// The k-th largest of n keys held by this CTA (keys[i * stride], i < n), by the
 // same MSB-first radix search as cluster_kth but with CTA barriers only:
 // the k largest keys are the keys > T plus the first `ties` keys == T in
 // index order.  1 <= k <= n.  sh.whist must be zero (it is left zero).
-template <int NT, class KeyAt>
-__device__ void cta_kth(KeyAt key_at, int n, int k, FinishShared& sh, uint32_t* T_out,
+template <int NT>
+__device__ __noinline__ void cta_kth(const uint32_t* keys, int stride, int n, int k,
+                                     FinishShared& sh, uint32_t* T_out,
                         int* ties_out) {
     constexpr int NW = NT / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint32_t kmin = 0xffffffffu, kmax = 0u;
     for (int i = tid; i < n; i += NT) {
-        const uint32_t v = key_at(i);
+        const uint32_t v = keys[i * stride];
         kmin = min(kmin, v);
         kmax = max(kmax, v);
     }
@@ -315,7 +315,7 @@ __device__ void cta_kth(KeyAt key_at, int n, int k, FinishShared& sh, uint32_t* 
         const int shift = max(hb - 7, 0);
         const uint32_t dmask = (1u << (hb - shift + 1)) - 1u;
         for (int i = tid; i < n; i += NT) {
-            const uint32_t v = key_at(i);
+            const uint32_t v = keys[i * stride];
             if ((v & mask) == prefix) atomicAdd(&wh[(v >> shift) & dmask], 1);
         }
         __syncthreads();
@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(FinishCfg<D>::NT, FinishCfg<D>::MIN_BLOCKS)
             if (bound) {
                 uint32_t tT;
                 int tties;
-                cta_kth<NT>([&](int i) { return tkeys[i]; }, ntiles, nsel, sh, &tT, &tties);
+                cta_kth<NT>(tkeys, 1, ntiles, nsel, sh, &tT, &tties);
                 const uint32_t tau = tties > 0 ? tT : tT + 1u;  // the nsel-th largest maximum
                 cp_async_wait<0>();  // this thread's phys[] copies
                 __syncthreads();     // every phys[] copy landed; tkeys is no longer read
@@ -514,8 +514,19 @@ __global__ void __launch_bounds__(FinishCfg<D>::NT, FinishCfg<D>::MIN_BLOCKS)
                     const bool keep = i < w1 && keys[i] >= tau;
                     const unsigned bk = __ballot_sync(0xffffffffu, keep);
                     const int pos = before + __popc(bk & below);
-                    if (keep && pos < kOwnSurvivorCap)
-                        own[pos] = Survivor{keys[i], c0 + i, phys[i], 0};
+                    if (keep && pos < kOwnSurvivorCap) {
+                        const int ph = phys[i];
+                        own[pos] = Survivor{keys[i], c0 + i, ph, 0};
+                        // every selected page is a survivor: its K and V start
+                        // their way into L2 now, while HBM idles through the
+                        // rest of the selection
+                        if (ph >= 0 && ph < a.num_pages) {
+                            constexpr uint32_t TILE = kPage * D * 2;
+                            const long long off = ((long long)ph * a.hkv + h) * TILE;
+                            prefetch_l2(static_cast<const uint8_t*>(a.k_cache) + off, TILE);
+                            prefetch_l2(static_cast<const uint8_t*>(a.v_cache) + off, TILE);
+                        }
+                    }
                     before += __popc(bk);
                 }
                 if (tid == 0) sh.scount = nown;
@@ -547,8 +558,7 @@ __global__ void __launch_bounds__(FinishCfg<D>::NT, FinishCfg<D>::MIN_BLOCKS)
                         __syncthreads();
                         uint32_t T;
                         int ties;
-                        cta_kth<NT>([&](int i) { return merged[i].key; }, total, nsel, sh, &T,
-                                    &ties);
+                        cta_kth<NT>(&merged[0].key, 4, total, nsel, sh, &T, &ties);
                         // the selected list: keys > T and the first `ties` keys == T,
                         // in index order (over the keys + phys area)
                         const int mspan = ((total + NW - 1) / NW + 31) / 32 * 32;
@@ -587,18 +597,6 @@ __global__ void __launch_bounds__(FinishCfg<D>::NT, FinishCfg<D>::MIN_BLOCKS)
                         // this CTA's share of selected_out
                         for (int i = rank + C * tid; i < p.budget; i += C * NT)
                             sel_row[i] = i < nsel ? list[i].x : -1;
-                        // the K and V of the pages this CTA attends start their way into L2
-                        constexpr uint32_t TILE = kPage * D * 2;
-                        for (int q = tid;; q += NT) {
-                            const int pp = (q / NW_ATT) * (C * NW_ATT) + rank * NW_ATT + q % NW_ATT;
-                            if (pp >= nsel) break;
-                            const int ph = list[pp].y;
-                            if (ph >= 0 && ph < a.num_pages) {
-                                const long long off = ((long long)ph * a.hkv + h) * TILE;
-                                prefetch_l2(static_cast<const uint8_t*>(a.k_cache) + off, TILE);
-                                prefetch_l2(static_cast<const uint8_t*>(a.v_cache) + off, TILE);
-                            }
-                        }
                         local_list = true;
                     }
                 }

@@ -74,6 +74,7 @@ struct KvAppendParams {
     const int32_t* positions;
     unsigned* status;
     int batch, hkv, max_pages, num_pages;
+    int meta_format;  // SLC_META_*
 };
 
 struct BuildMetaParams {
@@ -83,6 +84,7 @@ struct BuildMetaParams {
     const int32_t* seq_lens;
     unsigned* status;
     int batch, hkv, max_pages, num_pages;
+    int meta_format;  // SLC_META_*
 };
 
 struct ScoreParams {
@@ -97,6 +99,7 @@ struct ScoreParams {
     // (rows by candidate only, nullable) the largest order key (see
     // order_key) of each 16-candidate tile: [units][cand_stride / 16]
     uint32_t* tile_max;
+    int meta_format;  // SLC_META_*
 };
 
 struct SelectParams {

@@ -9,6 +9,10 @@
 //
 // min/max of bf16 values is a bf16 value, so the metadata is exact and the
 // incremental and rebuilt forms are bit-identical (up to the sign of zero).
+// E4M3 metadata (SLC_META_FP8_E4M3) stores the bounds rounded outward;
+// outward rounding is monotone, so min(round_down(a), round_down(b)) =
+// round_down(min(a, b)) and the incremental and rebuilt E4M3 bounds are
+// identical too.
 #include "slc_internal.h"
 
 namespace slc {
@@ -39,6 +43,34 @@ __device__ __forceinline__ uint4 shfl_xor4(uint4 v, int m) {
                       __shfl_xor_sync(0xffffffffu, v.z, m), __shfl_xor_sync(0xffffffffu, v.w, m));
 }
 
+// 8 bf16 (one 16-byte chunk) rounded outward to E4M3: 8 codes, low byte first.
+__device__ __forceinline__ uint2 round8(uint4 v, bool up) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t c[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float f = (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
+        c[i >> 2] |= e4m3_round(f, up) << (8 * (i & 3));
+    }
+    return make_uint2(c[0], c[1]);
+}
+
+// Bytewise min (up = false) or max (up = true) of two sets of 8 E4M3 codes,
+// by value.
+__device__ __forceinline__ uint2 pick8(uint2 a, uint2 b, bool up) {
+    const uint32_t wa[2] = {a.x, a.y}, wb[2] = {b.x, b.y};
+    uint32_t r[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t ca = (wa[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+        const uint32_t cb = (wb[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+        const float va = e4m3_value(ca), vb = e4m3_value(cb);
+        const uint32_t c = up ? (vb > va ? cb : ca) : (vb < va ? cb : ca);
+        r[i >> 2] |= c << (8 * (i & 3));
+    }
+    return make_uint2(r[0], r[1]);
+}
+
 // One warp per (sequence, kv head).  Chunk c < D/8 of the row is a 16-byte
 // piece of k, chunk c >= D/8 a piece of v.
 template <int D>
@@ -66,13 +98,19 @@ __global__ void __launch_bounds__(128) kv_append_kernel(KvAppendParams p) {
     const uint4* src_v = reinterpret_cast<const uint4*>(p.v_new) + ((long long)b * p.hkv + h) * CPR;
     uint4* dst_k = reinterpret_cast<uint4*>(p.k_cache) + (tile * kPage + slot) * CPR;
     uint4* dst_v = reinterpret_cast<uint4*>(p.v_cache) + (tile * kPage + slot) * CPR;
+    const bool fp8 = p.meta_format == SLC_META_FP8_E4M3;
     uint4* meta = reinterpret_cast<uint4*>(p.meta) + tile * 2 * CPR;
+    uint2* meta8 = reinterpret_cast<uint2*>(p.meta) + tile * 2 * CPR;  // [2][D] bytes
 #pragma unroll
     for (int c = lane; c < 2 * CPR; c += 32) {
         if (c < CPR) {
             const uint4 k = src_k[c];
             dst_k[c] = k;
-            if (slot == 0) {
+            if (fp8) {
+                const uint2 dn = round8(k, false), up = round8(k, true);
+                meta8[c] = slot == 0 ? dn : pick8(meta8[c], dn, false);
+                meta8[CPR + c] = slot == 0 ? up : pick8(meta8[CPR + c], up, true);
+            } else if (slot == 0) {
                 meta[c] = k;
                 meta[CPR + c] = k;
             } else {
@@ -127,6 +165,17 @@ __global__ void __launch_bounds__(256) build_meta_kernel(BuildMetaParams p) {
         if (RG == 2) {
             mn = min4(mn, shfl_xor4(mn, 16));
             mx = max4(mx, shfl_xor4(mx, 16));
+        }
+        if (p.meta_format == SLC_META_FP8_E4M3) {  // the bounds rounded outward
+            uint2* meta8 = reinterpret_cast<uint2*>(p.meta) + tile * 2 * CPR;
+            if (RG == 2) {
+                if (rg == 0) meta8[col] = round8(mn, false);
+                else meta8[CPR + col] = round8(mx, true);
+            } else {
+                meta8[col] = round8(mn, false);
+                meta8[CPR + col] = round8(mx, true);
+            }
+            continue;
         }
         uint4* meta = reinterpret_cast<uint4*>(p.meta) + tile * 2 * CPR;
         if (RG == 2) {

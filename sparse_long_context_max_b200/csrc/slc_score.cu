@@ -7,12 +7,11 @@
 //
 // Work split: tiles (16 consecutive candidate pages of one unit) of all
 // units are numbered in (b, h, tile) order and every warp of the
-// (persistent) grid takes a contiguous range of them (score_range in
+// (persistent) grid takes a contiguous range of them (score_range_bulk in
 // slc_score_impl.cuh).  Each warp streams its tiles through a private
-// shared-memory ring (two 8 KB tiles at D=128) filled by 16-byte
-// asynchronous copies, one cp.async group per tile.  Three 4-warp CTAs per
-// SM keep 24 tiles (192 KB) in flight.  The streaming kernel
-// (slc_stream.cu) runs the same range code after its prefix/window
+// shared-memory ring (two 8 KB tiles at D=128) filled by bulk copies.
+// Three 4-warp CTAs per SM keep 24 tiles (192 KB) in flight.  The streaming
+// kernel (slc_stream.cu) runs the same range code beside its prefix/window
 // attention.
 #include "slc_score_impl.cuh"
 
@@ -24,55 +23,71 @@ using namespace scr;
 
 constexpr int kScoreWarps = 4;  // warps per CTA
 
-template <int D>
-struct ScoreCfg : TileGeom<D> {
-    static constexpr int NT = D == 128 ? 2 : 1;  // tiles in flight per warp
-    static constexpr int RING_B = NT * TileGeom<D>::TILE_B;
-    static constexpr int SMEM = kScoreWarps * RING_B;  // 64 KB: three CTAs per SM
+// Ring per warp: two 8 KB tiles at D = 128 (bf16), one 16 KB tile at D =
+// 256; E4M3 tiles are half the size, so twice as many fit.
+template <int D, bool FP8>
+struct ScoreCfg {
+    static constexpr int NT = (D == 128 ? 2 : 1) * (FP8 ? 2 : 1);  // tiles in flight per warp
+    static constexpr int RING_B = NT * TileGeom<D, FP8>::TILE_B;
+    static constexpr int SMEM = kScoreWarps * (RING_B + NT * 8);    // 64 KB: three CTAs per SM
 };
 
-template <int D>
+template <int D, bool FP8>
 __global__ void __launch_bounds__(kScoreWarps * 32, 3) score_kernel(ScoreParams p) {
-    using C = ScoreCfg<D>;
+    using C = ScoreCfg<D, FP8>;
     extern __shared__ __align__(128) uint8_t smem[];
-    const int warp = threadIdx.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kScoreWarps * C::RING_B) + warp * C::NT;
+    if (lane == 0) {
+        for (int s = 0; s < C::NT; ++s) mbar_init(bars + s, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
     // inputs (q, metadata, lengths) may come from the preceding kernel
     grid_dep_wait();
     grid_dep_launch();
-    score_range<D, C::NT>(p, smem + warp * C::RING_B, blockIdx.x * kScoreWarps + warp,
-                          gridDim.x * kScoreWarps);
+    uint32_t it = 0;
+    score_range_bulk<D, C::NT, FP8>(p, smem + warp * C::RING_B, bars, it,
+                                    blockIdx.x * kScoreWarps + warp, gridDim.x * kScoreWarps);
+}
+
+template <int D, bool FP8>
+cudaError_t setup_one(int* occ) {
+    constexpr int smem = ScoreCfg<D, FP8>::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(score_kernel<D, FP8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, score_kernel<D, FP8>,
+                                                          kScoreWarps * 32, smem);
+    if (*occ < 1) *occ = 1;
+    return e;
+}
+
+template <int D, bool FP8>
+cudaError_t run(const ScoreParams& p, int occ, int num_sms, cudaStream_t stream) {
+    return launch_pdl(score_kernel<D, FP8>, dim3(num_sms * occ), dim3(kScoreWarps * 32),
+                      ScoreCfg<D, FP8>::SMEM, stream, 1, p);
 }
 
 }  // namespace
 
 cudaError_t setup_score(DeviceCfg& d) {
-    const int smem128 = ScoreCfg<128>::SMEM, smem256 = ScoreCfg<256>::SMEM;
-    cudaError_t e = cudaFuncSetAttribute(score_kernel<128>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem128);
-    if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_score[0], score_kernel<128>,
-                                                          kScoreWarps * 32, smem128);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(score_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 smem256);
-    if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_score[1], score_kernel<256>,
-                                                          kScoreWarps * 32, smem256);
-    for (int i = 0; i < 2; ++i)
-        if (d.occ_score[i] < 1) d.occ_score[i] = 1;
+    cudaError_t e = setup_one<128, false>(&d.occ_score[0]);
+    if (e == cudaSuccess) e = setup_one<256, false>(&d.occ_score[1]);
+    int occ;  // the E4M3 forms have the same shared memory: same occupancy
+    if (e == cudaSuccess) e = setup_one<128, true>(&occ);
+    if (e == cudaSuccess) e = setup_one<256, true>(&occ);
     return e;
 }
 
 cudaError_t launch_score(const ScoreParams& p, int head_dim, const DeviceCfg& d,
                          cudaStream_t stream) {
-    const bool d128 = head_dim == 128;
-    const int smem = d128 ? ScoreCfg<128>::SMEM : ScoreCfg<256>::SMEM;
-    const int blocks = d.num_sms * d.occ_score[d128 ? 0 : 1];
-    if (d128)
-        return launch_pdl(score_kernel<128>, dim3(blocks), dim3(kScoreWarps * 32), smem, stream,
-                          1, p);
-    return launch_pdl(score_kernel<256>, dim3(blocks), dim3(kScoreWarps * 32), smem, stream, 1,
-                      p);
+    const bool fp8 = p.meta_format == SLC_META_FP8_E4M3;
+    if (head_dim == 128)
+        return fp8 ? run<128, true>(p, d.occ_score[0], d.num_sms, stream)
+                   : run<128, false>(p, d.occ_score[0], d.num_sms, stream);
+    return fp8 ? run<256, true>(p, d.occ_score[1], d.num_sms, stream)
+               : run<256, false>(p, d.occ_score[1], d.num_sms, stream);
 }
 
 }  // namespace slc

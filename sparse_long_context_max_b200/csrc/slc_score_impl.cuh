@@ -12,12 +12,13 @@
 // two FMAs per metadata element whatever the group size.
 //
 // A tile is 16 consecutive candidate pages of one (sequence, kv head)
-// unit; one warp scores a tile held in shared memory (16 metadata rows of
-// 4*D bytes, in page order).  Lane l owns 16-byte chunks l, l+32, ... of
-// every row: it copies them itself (16-byte asynchronous copies, tracked by
-// its own cp.async groups) and dots them with its query weights; a
-// transposed butterfly (16 shuffles) then leaves page i's score in lanes
-// 2i and 2i+1.
+// unit; one warp scores a tile held in shared memory (16 metadata rows, in
+// page order, of 4*D bytes (bf16) or 2*D bytes (E4M3)), brought in by bulk
+// copies (TMA engine, one per page, issued by lanes 0..15) completing on
+// the ring stage's mbarrier.  Lane l owns chunks l, l+32, ... of every row
+// (16 bytes = 8 bf16, or 8 bytes = 8 E4M3: the same 8 dims either way) and
+// dots them with its query weights; a transposed butterfly (16 shuffles)
+// then leaves page i's score in lanes 2i and 2i+1.
 #pragma once
 
 #include "slc_internal.h"
@@ -27,12 +28,13 @@ namespace scr {
 
 constexpr int kTilePages = kSelTile;  // pages per tile (16)
 
-template <int D>
+template <int D, bool FP8 = false>
 struct TileGeom {
-    static constexpr int CPR = D / 8;                   // chunks per metadata row
+    static constexpr int CPR = D / 8;                   // chunks (8 dims) per metadata row
     static constexpr int CPL = 2 * CPR / 32;            // chunks per lane per page
-    static constexpr int PAGE_B = 4 * D;                // metadata bytes per (page, kv head)
-    static constexpr int TILE_B = kTilePages * PAGE_B;  // 8 KB / 16 KB
+    static constexpr int CHUNK_B = FP8 ? 8 : 16;        // bytes per chunk
+    static constexpr int PAGE_B = 2 * CPR * CHUNK_B;    // metadata bytes per (page, kv head)
+    static constexpr int TILE_B = kTilePages * PAGE_B;  // bf16 8 KB / 16 KB, E4M3 half
 };
 
 // 8 bf16 of a 16-byte chunk dotted with 8 fp32 weights: one unpack and one
@@ -46,6 +48,21 @@ __device__ __forceinline__ float dot8(const float (&w)[8], uint4 v) {
     s = fmaf(w[5], bf16_hi(v.z), s);
     s = fmaf(w[6], bf16_lo(v.w), s);
     s = fmaf(w[7], bf16_hi(v.w), s);
+    return s;
+}
+
+// 8 E4M3 codes (8 bytes, low byte first) dotted with 8 fp32 weights.
+__device__ __forceinline__ float dot8_e4m3(const float (&w)[8], uint2 v, float oor) {
+    const float2 a = e4m3x2_to_float2(v.x, oor), b = e4m3x2_to_float2(v.x >> 16, oor);
+    const float2 c = e4m3x2_to_float2(v.y, oor), d = e4m3x2_to_float2(v.y >> 16, oor);
+    float s = w[0] * a.x;
+    s = fmaf(w[1], a.y, s);
+    s = fmaf(w[2], b.x, s);
+    s = fmaf(w[3], b.y, s);
+    s = fmaf(w[4], c.x, s);
+    s = fmaf(w[5], c.y, s);
+    s = fmaf(w[6], d.x, s);
+    s = fmaf(w[7], d.y, s);
     return s;
 }
 
@@ -101,46 +118,32 @@ __device__ __forceinline__ int tile_phys(const ScoreParams& p, int u, const Page
     return phys;
 }
 
-// Copy the tile of kv head h whose page ids lane i < 16 holds (phys) into
-// dst (TILE_B bytes): for every page, lane l copies the 16-byte chunks l,
-// l+32, ... that it later reads itself.  Commits one cp.async group.
-template <int D>
-__device__ __forceinline__ void copy_tile(const ScoreParams& p, int h, int phys, uint8_t* dst) {
-    using C = TileGeom<D>;
-    const int lane = threadIdx.x & 31;
-    const uint8_t* src0 =
-        static_cast<const uint8_t*>(p.meta) + (long long)h * C::PAGE_B + lane * 16;
-    uint8_t* dst0 = dst + lane * 16;
-#pragma unroll
-    for (int pg = 0; pg < kTilePages; ++pg) {
-        const int ph = __shfl_sync(0xffffffffu, phys, pg);
-        if (ph >= 0) {
-            const uint8_t* src = src0 + (long long)ph * p.hkv * C::PAGE_B;
-#pragma unroll
-            for (int m = 0; m < C::CPL; ++m)
-                cp_async16(dst0 + pg * C::PAGE_B + m * 512, src + m * 512);
-        }
-    }
-    cp_async_commit();
-}
-
 // Score the landed tile jt of unit u (rows in `tile`) and write the page
 // scores; lane i < 16 holds page i's physical page in tphys (-1: the
 // block-table entry failed its check, and the page scores -inf).
-template <int D>
+template <int D, bool FP8>
 __device__ __forceinline__ void score_tile(const ScoreParams& p, int u, const PageRanges& r,
                                            int jt, const uint8_t* tile,
                                            const float (&w)[TileGeom<D>::CPL][8], int tphys) {
-    using C = TileGeom<D>;
+    using C = TileGeom<D, FP8>;
     const int lane = threadIdx.x & 31;
-    const uint8_t* t = tile + lane * 16;
+    const uint8_t* t = tile + lane * C::CHUNK_B;
     float acc[kTilePages];
 #pragma unroll
     for (int pg = 0; pg < kTilePages; ++pg) {
         float sacc = 0.f;
 #pragma unroll
-        for (int m = 0; m < C::CPL; ++m)
-            sacc += dot8(w[m], lds128(t + pg * C::PAGE_B + m * 512));
+        for (int m = 0; m < C::CPL; ++m) {
+            const uint8_t* src = t + pg * C::PAGE_B + m * 32 * C::CHUNK_B;
+            if (FP8) {
+                // kmin chunks (lane + 32m < CPR) read an out-of-range code as
+                // -kBf16Max, kmax chunks as +kBf16Max
+                const float oor = lane + 32 * m < C::CPR ? -kBf16Max : kBf16Max;
+                sacc += dot8_e4m3(w[m], lds64(src), oor);
+            } else {
+                sacc += dot8(w[m], lds128(src));
+            }
+        }
         acc[pg] = sacc;
     }
     __syncwarp();  // the caller may refill the tile's buffer after this
@@ -195,85 +198,16 @@ __device__ __forceinline__ void cursor_seek(const ScoreParams& p, TileCursor& c,
 
 // Score the tiles of warp gw of nw (tiles of all units numbered in (b, h,
 // tile) order, a contiguous range per warp) through this warp's ring of NT
-// tiles at `ring` (NT * TILE_B bytes).  The caller has waited for the
-// kernel that produces q, the metadata or the lengths.
-template <int D, int NT>
-__device__ void score_range(const ScoreParams& p, uint8_t* ring, int gw, int nw) {
-    using C = TileGeom<D>;
-    auto tiles_of = [&](int b) {
-        const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
-        const PageRanges r = page_ranges(L, p.prefix, p.window);
-        return (r.ws - r.np + kTilePages - 1) / kTilePages;
-    };
-    const int total = (int)total_units(p.batch, p.hkv, tiles_of);
-    const int per = (total + nw - 1) / nw;
-    const int g0 = gw * per;
-    const int g_end = min(total, g0 + per);
-    if (g0 >= g_end) return;
-
-    TileCursor use, iss;
-    {
-        long long us;
-        locate_unit(g0, p.batch, p.hkv, tiles_of, &use.u, &us);
-        use.ustart = (int)us;
-    }
-    cursor_seek(p, use, g0);
-    iss = use;
-    // issue side: tile gi is the next to copy; pf holds its page ids, loaded
-    // one copy ahead so the lookup overlaps the ring traffic.  Every call
-    // commits exactly one group (possibly empty) so that wait_group<NT-1>
-    // always means "the oldest tile has landed".
-    int gi = g0;
-    int pf = tile_phys(p, iss.u, iss.r, gi - iss.ustart);
-    int sp[NT];  // page ids of the tile in each slot (lane i: page i)
-    auto copy_next = [&](int slot) {
-        if (gi < g_end) {
-#pragma unroll
-            for (int k = 0; k < NT; ++k)
-                if (k == slot) sp[k] = pf;
-            copy_tile<D>(p, iss.u % p.hkv, pf, ring + slot * C::TILE_B);
-            ++gi;
-            if (gi < g_end) {
-                if (gi - iss.ustart >= iss.ntiles) cursor_seek(p, iss, gi);
-                pf = tile_phys(p, iss.u, iss.r, gi - iss.ustart);
-            }
-        } else {
-            cp_async_commit();
-        }
-    };
-#pragma unroll
-    for (int k = 0; k < NT; ++k) copy_next(k);
-
-    int wu = -1;  // unit whose weights are loaded
-    float w[C::CPL][8];
-    for (int g = g0; g < g_end; ++g) {
-        if (g - use.ustart >= use.ntiles) cursor_seek(p, use, g);
-        if (use.u != wu) {
-            wu = use.u;
-            load_weights<D>(p, use.u, w);
-        }
-        const int slot = (g - g0) % NT;
-        cp_async_wait<NT - 1>();  // this lane's chunks of the tile have landed
-        int tp = sp[0];
-#pragma unroll
-        for (int k = 1; k < NT; ++k)
-            if (k == slot) tp = sp[k];
-        score_tile<D>(p, use.u, use.r, g - use.ustart, ring + slot * C::TILE_B, w, tp);
-        copy_next(slot);  // refill: this lane's reads of the slot are done
-    }
-    cp_async_wait<0>();
-}
-
-// score_range with the tiles brought in by bulk copies (TMA engine, one per
-// page row of 4*D bytes, issued by lanes 0..15) completing on the ring
-// stage's mbarrier, instead of per-lane 16-byte copies: the streaming
-// kernel's form.  bars: NT mbarriers (count 1) whose next phase parity is
+// tiles at `ring` (NT * TILE_B bytes), each filled by bulk copies completing
+// on its mbarrier.  bars: NT mbarriers (count 1) whose next phase parity is
 // `it` (ring uses so far, advanced here).  A bounded wait that gives up sets
-// SLC_STATUS_WAIT_TIMEOUT; the warp then drains its copies and stops.
-template <int D, int NT>
+// SLC_STATUS_WAIT_TIMEOUT; the warp then drains its copies and stops.  The
+// caller has waited for the kernel that produces q, the metadata or the
+// lengths.
+template <int D, int NT, bool FP8>
 __device__ void score_range_bulk(const ScoreParams& p, uint8_t* ring, uint64_t* bars,
                                  uint32_t& it, int gw, int nw) {
-    using C = TileGeom<D>;
+    using C = TileGeom<D, FP8>;
     const int lane = threadIdx.x & 31;
     auto tiles_of = [&](int b) {
         const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
@@ -350,7 +284,7 @@ __device__ void score_range_bulk(const ScoreParams& p, uint8_t* ring, uint64_t* 
 #pragma unroll
         for (int k = 1; k < NT; ++k)
             if (k == slot) tp = sp[k];
-        score_tile<D>(p, use.u, use.r, g - use.ustart, ring + slot * C::TILE_B, w, tp);
+        score_tile<D, FP8>(p, use.u, use.r, g - use.ustart, ring + slot * C::TILE_B, w, tp);
         fence_proxy_async_smem();  // this warp's reads of the slot precede its refill
         copy_next(slot);
     }

@@ -29,24 +29,28 @@ struct StreamCfg {
     static constexpr int NW = 4;                   // warps per CTA
     static constexpr int STAGES = D == 128 ? 2 : 3;  // ring stages per warp
     static constexpr int RING = STAGES * 2 * kPage * D * 2;
-    static constexpr int SMEM = NW * STAGES * (2 * kPage * D * 2 + 8 + 4);
+    // a K+V page stage holds one bf16 metadata tile or two E4M3 tiles; the
+    // ring has an mbarrier for each of the latter
+    static constexpr int NBAR = 2 * STAGES;
+    static constexpr int SMEM = NW * (RING + NBAR * 8 + STAGES * 4);
     static constexpr int MIN_BLOCKS = D == 128 ? 3 : 1;
 };
 
-template <int D>
+template <int D, bool FP8>
 __global__ void __launch_bounds__(StreamCfg<D>::NW * 32, StreamCfg<D>::MIN_BLOCKS)
     stream_kernel(StreamParams p) {
     using C = StreamCfg<D>;
     static_assert(C::RING == C::STAGES * scr::TileGeom<D>::TILE_B, "ring holds NT tiles");
+    static_assert(C::RING == C::NBAR * scr::TileGeom<D, true>::TILE_B, "or 2 NT E4M3 tiles");
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     Ring ring;
     ring.tiles = smem + warp * C::RING;
-    ring.bars = reinterpret_cast<uint64_t*>(smem + C::NW * C::RING) + warp * C::STAGES;
+    ring.bars = reinterpret_cast<uint64_t*>(smem + C::NW * C::RING) + warp * C::NBAR;
     ring.nvalid =
-        reinterpret_cast<int*>(smem + C::NW * C::RING + C::NW * C::STAGES * 8) + warp * C::STAGES;
+        reinterpret_cast<int*>(smem + C::NW * C::RING + C::NW * C::NBAR * 8) + warp * C::STAGES;
     if (lane == 0) {
-        for (int s = 0; s < C::STAGES; ++s) mbar_init(ring.bars + s, 1);
+        for (int s = 0; s < C::NBAR; ++s) mbar_init(ring.bars + s, 1);
         fence_mbar_init();
     }
     __syncwarp();
@@ -70,29 +74,42 @@ __global__ void __launch_bounds__(StreamCfg<D>::NW * 32, StreamCfg<D>::MIN_BLOCK
     } else if (p.sc.scores != nullptr) {
         // candidate scores, tiles spread over the remaining CTAs' warps
         uint32_t it = 0;
-        scr::score_range_bulk<D, C::STAGES>(p.sc, ring.tiles, ring.bars, it,
-                                            (blockIdx.x - nf) * C::NW + warp,
-                                            (gridDim.x - nf) * C::NW);
+        scr::score_range_bulk<D, FP8 ? C::NBAR : C::STAGES, FP8>(
+            p.sc, ring.tiles, ring.bars, it, (blockIdx.x - nf) * C::NW + warp,
+            (gridDim.x - nf) * C::NW);
     }
 }
 
-template <int D>
+template <int D, bool FP8>
 cudaError_t setup_one(int* occ) {
-    cudaError_t e = cudaFuncSetAttribute(stream_kernel<D>,
+    cudaError_t e = cudaFuncSetAttribute(stream_kernel<D, FP8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          StreamCfg<D>::SMEM);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, stream_kernel<D>,
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, stream_kernel<D, FP8>,
                                                       StreamCfg<D>::NW * 32, StreamCfg<D>::SMEM);
     if (*occ < 1) *occ = 1;
     return e;
 }
 
+template <int D, bool FP8>
+cudaError_t run(StreamParams& p, int blocks, cudaStream_t stream) {
+    return launch_pdl(stream_kernel<D, FP8>, dim3(blocks), dim3(StreamCfg<D>::NW * 32),
+                      StreamCfg<D>::SMEM, stream, 1, p);
+}
+
 }  // namespace
 
 cudaError_t setup_stream(DeviceCfg& d) {
-    cudaError_t e = setup_one<128>(&d.occ_stream[0]);
-    if (e == cudaSuccess) e = setup_one<256>(&d.occ_stream[1]);
+    // one occupancy per head_dim: the E4M3 forms use the same resources
+    // (the grid size, hence the chunk count, must not depend on the format)
+    cudaError_t e = setup_one<128, false>(&d.occ_stream[0]);
+    if (e == cudaSuccess) e = setup_one<256, false>(&d.occ_stream[1]);
+    int occ;
+    if (e == cudaSuccess) e = setup_one<128, true>(&occ);
+    if (e == cudaSuccess && occ < d.occ_stream[0]) d.occ_stream[0] = occ;
+    if (e == cudaSuccess) e = setup_one<256, true>(&occ);
+    if (e == cudaSuccess && occ < d.occ_stream[1]) d.occ_stream[1] = occ;
     return e;
 }
 
@@ -107,11 +124,9 @@ cudaError_t launch_stream(StreamParams& p, int head_dim, const DeviceCfg& d,
     const int blocks = stream_chunks(head_dim, d);
     p.at.num_chunks = blocks;
     p.at.list = kListForced;
-    if (d128)
-        return launch_pdl(stream_kernel<128>, dim3(blocks), dim3(StreamCfg<128>::NW * 32),
-                          StreamCfg<128>::SMEM, stream, 1, p);
-    return launch_pdl(stream_kernel<256>, dim3(blocks), dim3(StreamCfg<256>::NW * 32),
-                      StreamCfg<256>::SMEM, stream, 1, p);
+    const bool fp8 = p.sc.meta_format == SLC_META_FP8_E4M3;
+    if (d128) return fp8 ? run<128, true>(p, blocks, stream) : run<128, false>(p, blocks, stream);
+    return fp8 ? run<256, true>(p, blocks, stream) : run<256, false>(p, blocks, stream);
 }
 
 }  // namespace slc

@@ -12,7 +12,7 @@ TIE_BAND = 1e-4  # selections may differ only on pages this close to the k-th sc
 class Dev:
     """Device copies of one layer's inputs, plus the cache object."""
 
-    def __init__(self, x, build_meta=True):
+    def __init__(self, x, build_meta=True, meta_format="bf16"):
         import sparse_long_context_max_b200 as slc
         self.x = x
         self.q = x.q.cuda()
@@ -20,7 +20,8 @@ class Dev:
         self.v = x.v_cache.cuda()
         self.bt = x.block_table.cuda()
         self.sl = x.seq_lens.cuda()
-        self.cache = slc.PagedCache(self.k, self.v)
+        self.meta_format = meta_format
+        self.cache = slc.PagedCache(self.k, self.v, meta_format=meta_format)
         if build_meta:
             slc.build_page_meta(self.cache, self.bt, self.sl)
 
@@ -47,13 +48,23 @@ class Dev:
         return out.cpu().double().numpy()
 
 
-def check_selection(x, sel_gpu, prefix, window, budget, scores=None):
+def oracle_scores(x, prefix, window, meta_format="bf16"):
+    """The oracle's page scores from bf16 bounds, or from the E4M3 bounds
+    rounded outward."""
+    if meta_format == "fp8":
+        c8min, c8max = oracle.page_bounds_fp8(x.k_cache, x.block_table, x.seq_lens)
+        kmin, kmax = oracle.fp8_decode(c8min), oracle.fp8_decode(c8max)
+    else:
+        kmin, kmax = oracle.page_bounds(x.k_cache, x.block_table, x.seq_lens)
+    return oracle.page_scores(x.q, kmin, kmax, x.seq_lens, prefix, window)
+
+
+def check_selection(x, sel_gpu, prefix, window, budget, scores=None, meta_format="bf16"):
     """GPU selection == oracle selection, except pages whose oracle score is
     within TIE_BAND (relative) of the k-th oracle score.  Returns the oracle
     selection."""
     if scores is None:
-        kmin, kmax = oracle.page_bounds(x.k_cache, x.block_table, x.seq_lens)
-        scores = oracle.page_scores(x.q, kmin, kmax, x.seq_lens, prefix, window)
+        scores = oracle_scores(x, prefix, window, meta_format)
     sel_o, nsel_o = oracle.select_pages(scores, x.seq_lens, prefix, window, budget)
     B, hkv, _ = sel_o.shape
     for b in range(B):

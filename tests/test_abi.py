@@ -63,7 +63,7 @@ FAKE = 0x10000  # a 16-byte aligned address that is never dereferenced
 
 def cache(**kw):
     c = dict(k_cache=FAKE, v_cache=FAKE, meta=FAKE, num_pages=10, num_kv_heads=2,
-             head_dim=128, page_size=16)
+             head_dim=128, page_size=16, meta_format=0)
     c.update(kw)
     return slc._Cache(**c)
 
@@ -81,6 +81,7 @@ def sparse(c, q=FAKE, hq=8, batch=1, max_pages=10, prefix=0, window=0, budget=2,
     (dict(num_pages=0), INVALID),
     (dict(k_cache=None), INVALID),
     (dict(meta=FAKE + 8), INVALID),  # misaligned
+    (dict(meta_format=2), UNSUPPORTED),  # no such metadata format
 ])
 def test_cache_validation(kw, code):
     assert sparse(cache(**kw)) == code

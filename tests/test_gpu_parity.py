@@ -9,7 +9,8 @@ import torch
 
 import oracle
 import synth
-from gpu_util import (Dev, check_needles, check_output, check_selection, slice_batch)
+from gpu_util import (Dev, check_needles, check_output, check_selection, oracle_scores,
+                      slice_batch)
 
 pytestmark = pytest.mark.gpu
 
@@ -523,3 +524,75 @@ def test_layers131k_graph_step_all_layers():
         check_output(y, out, wl.prefix, s.window, sel)
     del caches, step
     torch.cuda.empty_cache()
+
+
+
+# ------------------------------------------------------------------ E4M3 metadata
+
+def meta8_matches_oracle(d):
+    """The device's E4M3 bounds equal the oracle's outward-rounded codes,
+    bit for bit."""
+    x = d.x
+    c8min, c8max = oracle.page_bounds_fp8(x.k_cache, x.block_table, x.seq_lens)
+    meta = d.cache.meta.cpu().numpy()  # uint8 [pages][Hkv][2][D]
+    bt = x.block_table.numpy()
+    for b, L in enumerate(x.seq_lens.tolist()):
+        n = -(-L // 16)
+        phys = bt[b, :n]
+        np.testing.assert_array_equal(meta[phys, :, 0, :].transpose(1, 0, 2), c8min[b, :, :n])
+        np.testing.assert_array_equal(meta[phys, :, 1, :].transpose(1, 0, 2), c8max[b, :, :n])
+
+
+@pytest.mark.parametrize("hq,hkv,D", [(8, 2, 128), (16, 2, 256)])
+def test_fp8_meta_build_and_append_exact(hq, hkv, D):
+    """E4M3 metadata, built and appended: bit-exact against the oracle's
+    outward rounding, keys spread from subnormal E4M3 to beyond +-448 and
+    NaN/Inf in unused slots; the appended form equals a rebuild."""
+    import sparse_long_context_max_b200 as slc
+    x = small(3, hq, hkv, D, [30, 47, 16], seed=23 + D, headroom=40, fill="nan")
+    g = torch.Generator().manual_seed(5)
+    scale = torch.exp(torch.randn(x.k_cache.shape, generator=g) * 3)  # e^-9 .. e^9
+    x.k_cache = torch.where(torch.isfinite(x.k_cache.float()),
+                            x.k_cache.float() * scale, x.k_cache.float()).to(torch.bfloat16)
+    d = Dev(x, meta_format="fp8")
+    meta8_matches_oracle(d)
+    lens = x.seq_lens.clone()
+    for step in range(40):
+        kn = (torch.randn((3, hkv, D), generator=torch.Generator().manual_seed(step)) *
+              torch.exp(torch.randn((3, hkv, D), generator=g) * 3)).to(torch.bfloat16)
+        vn = torch.randn((3, hkv, D), generator=torch.Generator().manual_seed(77 + step)).to(torch.bfloat16)
+        slc.kv_append(d.cache, kn.cuda(), vn.cuda(), d.bt, lens.cuda())
+        for b in range(3):
+            L = int(lens[b])
+            phys = int(x.block_table[b, L // 16])
+            x.k_cache[phys, :, L % 16] = kn[b]
+            x.v_cache[phys, :, L % 16] = vn[b]
+        lens += 1
+    torch.cuda.synchronize()
+    assert slc.device_status() == 0
+    x.seq_lens = lens
+    d.sl = lens.cuda()
+    incremental = d.cache.meta.clone()
+    meta8_matches_oracle(d)
+    slc.build_page_meta(d.cache, d.bt, d.sl)
+    used = sorted(set(int(p) for b in range(3) for p in x.block_table[b, : -(-int(lens[b]) // 16)]))
+    assert torch.equal(incremental[used], d.cache.meta[used])
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode256k"])
+def test_fp8_meta_decode_parity(name):
+    """Sparse decode over E4M3 metadata: the decode path's own scores against
+    the oracle's scores from the outward-rounded bounds (2e-6 relative), the
+    selection within the tie band of those scores, the output against the
+    oracle attending the GPU's selection, and needles still selected."""
+    x = synth.make_inputs(W[name])
+    d = Dev(x, meta_format="fp8")
+    so = oracle_scores(x, x.prefix, x.window, "fp8")
+    s = stream_scores(d, x.prefix, x.window, x.budget)
+    cand = ~np.isnan(so)
+    assert (np.isnan(s) == ~cand).all()
+    assert np.abs(s[cand] - so[cand]).max() <= 2e-6 * np.abs(so[cand]).max()
+    out, sel = d.sparse()
+    check_selection(x, sel, x.prefix, x.window, x.budget, scores=so)
+    check_needles(x, sel)
+    check_output(x, out, x.prefix, x.window, sel)
