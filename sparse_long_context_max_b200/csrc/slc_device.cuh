@@ -244,6 +244,19 @@ __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
                  : "memory");
 }
 
+// 16- or 8-byte asynchronous global -> shared copy (both aligned to its
+// size); 16-byte copies bypass L1.
+template <int B>
+__device__ __forceinline__ void cp_async_chunk(void* dst, const void* src) {
+    static_assert(B == 16 || B == 8, "16- or 8-byte copies");
+    if (B == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
+                     : "memory");
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_addr(dst)), "l"(src)
+                     : "memory");
+}
+
 __device__ __forceinline__ void cp_async_commit() {
     asm volatile("cp.async.commit_group;" ::: "memory");
 }

@@ -7,12 +7,11 @@
 //
 // Work split: tiles (16 consecutive candidate pages of one unit) of all
 // units are numbered in (b, h, tile) order and every warp of the
-// (persistent) grid takes a contiguous range of them (score_range_bulk in
-// slc_score_impl.cuh).  Each warp streams its tiles through a private
-// shared-memory ring (two 8 KB tiles at D=128) filled by bulk copies.
-// Three 4-warp CTAs per SM keep 24 tiles (192 KB) in flight.  The streaming
-// kernel (slc_stream.cu) runs the same range code beside its prefix/window
-// attention.
+// (persistent) grid takes a contiguous range of them.  Each warp streams its
+// tiles through a private shared-memory ring (two 8 KB tiles at D=128)
+// filled by asynchronous copies (score_run in slc_score_impl.cuh).  Three
+// 4-warp CTAs per SM keep 24 tiles (192 KB) in flight.  The sparse decode
+// kernel (slc_decode.cu) scores with the same code.
 #include "slc_score_impl.cuh"
 
 namespace slc {
@@ -29,26 +28,47 @@ template <int D, bool FP8>
 struct ScoreCfg {
     static constexpr int NT = (D == 128 ? 2 : 1) * (FP8 ? 2 : 1);  // tiles in flight per warp
     static constexpr int RING_B = NT * TileGeom<D, FP8>::TILE_B;
-    static constexpr int SMEM = kScoreWarps * (RING_B + NT * 8);    // 64 KB: three CTAs per SM
+    static constexpr int SMEM = kScoreWarps * RING_B;               // 64 KB: three CTAs per SM
 };
 
 template <int D, bool FP8>
 __global__ void __launch_bounds__(kScoreWarps * 32, 3) score_kernel(ScoreParams p) {
     using C = ScoreCfg<D, FP8>;
     extern __shared__ __align__(128) uint8_t smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kScoreWarps * C::RING_B) + warp * C::NT;
-    if (lane == 0) {
-        for (int s = 0; s < C::NT; ++s) mbar_init(bars + s, 1);
-        fence_mbar_init();
-    }
-    __syncwarp();
+    const int warp = threadIdx.x >> 5;
     // inputs (q, metadata, lengths) may come from the preceding kernel
     grid_dep_wait();
     grid_dep_launch();
-    uint32_t it = 0;
-    score_range_bulk<D, C::NT, FP8>(p, smem + warp * C::RING_B, bars, it,
-                                    blockIdx.x * kScoreWarps + warp, gridDim.x * kScoreWarps);
+    auto tiles_of = [&](int b) {
+        const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
+        const PageRanges r = page_ranges(L, p.prefix, p.window);
+        return (r.ws - r.np + kTilePages - 1) / kTilePages;
+    };
+    const long long total = total_units(p.batch, p.hkv, tiles_of);
+    const long long nw = (long long)gridDim.x * kScoreWarps;
+    const long long per = (total + nw - 1) / nw;
+    long long g = ((long long)blockIdx.x * kScoreWarps + warp) * per;
+    const long long g_end = min(total, g + per);
+    if (g >= g_end) return;
+    int u;
+    long long ustart;
+    locate_unit(g, p.batch, p.hkv, tiles_of, &u, &ustart);
+    // the units this warp's range crosses, in order
+    while (g < g_end && u < p.batch * p.hkv) {
+        const int L = checked_len(p.seq_lens, u / p.hkv, p.max_pages, p.status);
+        const PageRanges r = page_ranges(L, p.prefix, p.window);
+        const long long uend = ustart + (r.ws - r.np + kTilePages - 1) / kTilePages;
+        const long long stop = min(g_end, uend);
+        if (stop > g) {
+            float w[TileGeom<D>::CPL][8];
+            load_weights<D>(p, u, w);
+            score_run<D, C::NT, FP8>(p, smem + warp * C::RING_B, u, r, (int)(g - ustart),
+                                     (int)(stop - ustart), w);
+            g = stop;
+        }
+        ustart = uend;
+        ++u;
+    }
 }
 
 template <int D, bool FP8>

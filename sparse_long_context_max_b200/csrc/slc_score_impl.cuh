@@ -13,12 +13,13 @@
 //
 // A tile is 16 consecutive candidate pages of one (sequence, kv head)
 // unit; one warp scores a tile held in shared memory (16 metadata rows, in
-// page order, of 4*D bytes (bf16) or 2*D bytes (E4M3)), brought in by bulk
-// copies (TMA engine, one per page, issued by lanes 0..15) completing on
-// the ring stage's mbarrier.  Lane l owns chunks l, l+32, ... of every row
-// (16 bytes = 8 bf16, or 8 bytes = 8 E4M3: the same 8 dims either way) and
-// dots them with its query weights; a transposed butterfly (16 shuffles)
-// then leaves page i's score in lanes 2i and 2i+1.
+// page order, of 4*D bytes (bf16) or 2*D bytes (E4M3)), brought in by
+// asynchronous 16- or 8-byte copies (score_run).  Lane l owns chunks l,
+// l+32, ... of every row (16 bytes = 8 bf16, or 8 bytes = 8 E4M3: the same
+// 8 dims either way) and dots them with its query weights; a transposed
+// butterfly (16 shuffles) then leaves page i's score in lanes 2i and 2i+1.
+// (Per-page bulk copies through the TMA engine were measured slower here:
+// 512-byte copies cap the read rate well below the HBM rate.)
 #pragma once
 
 #include "slc_internal.h"
@@ -37,33 +38,25 @@ struct TileGeom {
     static constexpr int TILE_B = kTilePages * PAGE_B;  // bf16 8 KB / 16 KB, E4M3 half
 };
 
-// 8 bf16 of a 16-byte chunk dotted with 8 fp32 weights: one unpack and one
-// FMA per element.
+// 8 bf16 of a 16-byte chunk dotted with 8 fp32 weights: one unpack per
+// element and one packed two-lane FMA per pair.
 __device__ __forceinline__ float dot8(const float (&w)[8], uint4 v) {
-    float s = w[0] * bf16_lo(v.x);
-    s = fmaf(w[1], bf16_hi(v.x), s);
-    s = fmaf(w[2], bf16_lo(v.y), s);
-    s = fmaf(w[3], bf16_hi(v.y), s);
-    s = fmaf(w[4], bf16_lo(v.z), s);
-    s = fmaf(w[5], bf16_hi(v.z), s);
-    s = fmaf(w[6], bf16_lo(v.w), s);
-    s = fmaf(w[7], bf16_hi(v.w), s);
-    return s;
+    float2 s = make_float2(bf16_lo(v.x) * w[0], bf16_hi(v.x) * w[1]);
+    s = ffma2(make_float2(bf16_lo(v.y), bf16_hi(v.y)), make_float2(w[2], w[3]), s);
+    s = ffma2(make_float2(bf16_lo(v.z), bf16_hi(v.z)), make_float2(w[4], w[5]), s);
+    s = ffma2(make_float2(bf16_lo(v.w), bf16_hi(v.w)), make_float2(w[6], w[7]), s);
+    return s.x + s.y;
 }
 
 // 8 E4M3 codes (8 bytes, low byte first) dotted with 8 fp32 weights.
 __device__ __forceinline__ float dot8_e4m3(const float (&w)[8], uint2 v, float oor) {
     const float2 a = e4m3x2_to_float2(v.x, oor), b = e4m3x2_to_float2(v.x >> 16, oor);
     const float2 c = e4m3x2_to_float2(v.y, oor), d = e4m3x2_to_float2(v.y >> 16, oor);
-    float s = w[0] * a.x;
-    s = fmaf(w[1], a.y, s);
-    s = fmaf(w[2], b.x, s);
-    s = fmaf(w[3], b.y, s);
-    s = fmaf(w[4], c.x, s);
-    s = fmaf(w[5], c.y, s);
-    s = fmaf(w[6], d.x, s);
-    s = fmaf(w[7], d.y, s);
-    return s;
+    float2 s = make_float2(a.x * w[0], a.y * w[1]);
+    s = ffma2(b, make_float2(w[2], w[3]), s);
+    s = ffma2(c, make_float2(w[4], w[5]), s);
+    s = ffma2(d, make_float2(w[6], w[7]), s);
+    return s.x + s.y;
 }
 
 // Group-reduced query weights of this lane's chunks of unit u: chunk
@@ -177,118 +170,67 @@ __device__ __forceinline__ void score_tile(const ScoreParams& p, int u, const Pa
 }
 
 
-// Cursor over the tiles of consecutive units.
-struct TileCursor {
-    int u;
-    int ustart;  // global index of the unit's first tile
-    int ntiles;  // tiles of unit u
-    PageRanges r;
-};
-
-__device__ __forceinline__ void cursor_seek(const ScoreParams& p, TileCursor& c, int g) {
-    while (true) {
-        const int L = checked_len(p.seq_lens, c.u / p.hkv, p.max_pages, p.status);
-        c.r = page_ranges(L, p.prefix, p.window);
-        c.ntiles = (c.r.ws - c.r.np + kTilePages - 1) / kTilePages;
-        if (g - c.ustart < c.ntiles) return;
-        c.ustart += c.ntiles;
-        ++c.u;
-    }
-}
-
-// Score the tiles of warp gw of nw (tiles of all units numbered in (b, h,
-// tile) order, a contiguous range per warp) through this warp's ring of NT
-// tiles at `ring` (NT * TILE_B bytes), each filled by bulk copies completing
-// on its mbarrier.  bars: NT mbarriers (count 1) whose next phase parity is
-// `it` (ring uses so far, advanced here).  A bounded wait that gives up sets
-// SLC_STATUS_WAIT_TIMEOUT; the warp then drains its copies and stops.  The
-// caller has waited for the kernel that produces q, the metadata or the
-// lengths.
-template <int D, int NT, bool FP8>
-__device__ void score_range_bulk(const ScoreParams& p, uint8_t* ring, uint64_t* bars,
-                                 uint32_t& it, int gw, int nw) {
+// Score tiles [j0, j1) of unit u (page ranges r) with this warp, through
+// its ring of NS tiles at `ring` (NS * TILE_B bytes).  Every lane copies its
+// own chunks of each page (asynchronous 16- or 8-byte copies: one warp
+// instruction moves one page's row, fully coalesced), one copy group per
+// tile, NS tiles in flight; each lane reads back only the chunks it copied.
+// (Copies that give each lane a contiguous half row take one shuffle per
+// tile instead of sixteen but coalesce worse, and measured slower.)  w: the
+// unit's query weights (load_weights).  The caller has waited for the kernel
+// that produces q, the metadata or the lengths, and nothing else writes the
+// ring meanwhile.
+template <int D, int NS, bool FP8>
+__device__ void score_run(const ScoreParams& p, uint8_t* ring, int u, const PageRanges& r,
+                          int j0, int j1, const float (&w)[TileGeom<D>::CPL][8]) {
     using C = TileGeom<D, FP8>;
     const int lane = threadIdx.x & 31;
-    auto tiles_of = [&](int b) {
-        const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
-        const PageRanges r = page_ranges(L, p.prefix, p.window);
-        return (r.ws - r.np + kTilePages - 1) / kTilePages;
-    };
-    const int total = (int)total_units(p.batch, p.hkv, tiles_of);
-    const int per = (total + nw - 1) / nw;
-    const int g0 = gw * per;
-    const int g_end = min(total, g0 + per);
-    if (g0 >= g_end) return;
-
-    TileCursor use, iss;
-    {
-        long long us;
-        locate_unit(g0, p.batch, p.hkv, tiles_of, &use.u, &us);
-        use.ustart = (int)us;
-    }
-    cursor_seek(p, use, g0);
-    iss = use;
-    int gi = g0;
-    int pf = tile_phys(p, iss.u, iss.r, gi - iss.ustart);
-    int sp[NT];  // page ids of the tile in each slot (lane i: page i)
-    const uint8_t* meta = static_cast<const uint8_t*>(p.meta);
-    // issue tile gi into stage `slot` (page ids in pf), then look one tile ahead
-    auto copy_next = [&](int slot) {
-        if (gi >= g_end) return;
+    const int n = j1 - j0;
+    if (n <= 0) return;
+    const uint8_t* meta = static_cast<const uint8_t*>(p.meta) +
+                          (long long)(u % p.hkv) * C::PAGE_B + lane * C::CHUNK_B;
+    const long long page_stride = (long long)p.hkv * C::PAGE_B;
+    int pf = tile_phys(p, u, r, j0);  // lane i < 16: page i of the next tile to copy
+    int sp[NS];                       // the same for the tile in each slot
 #pragma unroll
-        for (int k = 0; k < NT; ++k)
-            if (k == slot) sp[k] = pf;
-        const unsigned have = __ballot_sync(0xffffffffu, pf >= 0);
-        if (lane == 0) {
-            if (have) mbar_arrive_expect_tx(bars + slot, __popc(have) * C::PAGE_B);
-            else mbar_arrive(bars + slot);
-        }
-        __syncwarp();
-        if (pf >= 0) {
-            const long long src = ((long long)pf * p.hkv + iss.u % p.hkv) * C::PAGE_B;
-            bulk_g2s(ring + slot * C::TILE_B + lane * C::PAGE_B, meta + src, C::PAGE_B,
-                     bars + slot);
-        }
-        ++gi;
-        if (gi < g_end) {
-            if (gi - iss.ustart >= iss.ntiles) cursor_seek(p, iss, gi);
-            pf = tile_phys(p, iss.u, iss.r, gi - iss.ustart);
-        }
-    };
-    fence_proxy_async_smem();  // earlier generic accesses of the ring first
+    for (int k = 0; k < NS; ++k) sp[k] = -1;
+    // copy tile j0 + k into slot k % NS (nothing past the range), then look
+    // one tile ahead; always one commit, so group k is tile k
+    auto issue = [&](int k) {
+        if (k < n) {
+            const int slot = k % NS;
 #pragma unroll
-    for (int k = 0; k < NT; ++k) copy_next((it + k) % NT);
-
-    int wu = -1;  // unit whose weights are loaded
-    float w[C::CPL][8];
-    for (int g = g0; g < g_end; ++g) {
-        if (g - use.ustart >= use.ntiles) cursor_seek(p, use, g);
-        if (use.u != wu) {
-            wu = use.u;
-            load_weights<D>(p, use.u, w);
-        }
-        const uint32_t u_ = it + (g - g0);
-        const int slot = u_ % NT;
-        if (!mbar_wait_bounded(bars + slot, (u_ / NT) & 1u, 1u << 22)) {
-            if (lane == 0) {
-                atomicOr(p.status, SLC_STATUS_WAIT_TIMEOUT);
-                for (int k = g + 1; k < g_end && k < g + NT; ++k) {
-                    const uint32_t u2 = it + (k - g0);
-                    mbar_wait_bounded(bars + u2 % NT, (u2 / NT) & 1u, 1u << 22);
+            for (int s2 = 0; s2 < NS; ++s2)
+                if (s2 == slot) sp[s2] = pf;
+            uint8_t* dst = ring + slot * C::TILE_B + lane * C::CHUNK_B;
+#pragma unroll
+            for (int pg = 0; pg < kTilePages; ++pg) {
+                const int ph = __shfl_sync(0xffffffffu, pf, pg);
+                if (ph >= 0) {
+                    const uint8_t* src = meta + ph * page_stride;
+#pragma unroll
+                    for (int m = 0; m < C::CPL; ++m)
+                        cp_async_chunk<C::CHUNK_B>(dst + pg * C::PAGE_B + m * 32 * C::CHUNK_B,
+                                                   src + m * 32 * C::CHUNK_B);
                 }
             }
-            __syncwarp();
-            return;
+            if (k + 1 < n) pf = tile_phys(p, u, r, j0 + k + 1);
         }
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int k = 0; k < NS; ++k) issue(k);
+    for (int k = 0; k < n; ++k) {
+        cp_async_wait<NS - 1>();  // tile k (this lane's chunks) has landed
+        const int slot = k % NS;
         int tp = sp[0];
 #pragma unroll
-        for (int k = 1; k < NT; ++k)
-            if (k == slot) tp = sp[k];
-        score_tile<D, FP8>(p, use.u, use.r, g - use.ustart, ring + slot * C::TILE_B, w, tp);
-        fence_proxy_async_smem();  // this warp's reads of the slot precede its refill
-        copy_next(slot);
+        for (int s2 = 1; s2 < NS; ++s2)
+            if (s2 == slot) tp = sp[s2];
+        score_tile<D, FP8>(p, u, r, j0 + k, ring + slot * C::TILE_B, w, tp);
+        issue(k + NS);
     }
-    it += g_end - g0;
+    cp_async_wait<0>();
 }
 
 }  // namespace scr

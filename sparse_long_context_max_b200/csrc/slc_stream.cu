@@ -8,7 +8,8 @@
 //     like the dense kernel's (slot = unit + chunk, the forced lists of all
 //     units concatenated and cut into one chunk per attending CTA);
 //   - the Quest bound of every candidate page (same section), written by
-//     candidate into 16-byte aligned rows, as score_kernel does.
+//     candidate into 16-byte aligned rows, as score_kernel does, with the
+//     same per-warp copy pipeline (score_run in slc_score_impl.cuh).
 //
 // The two run side by side: the first CTAs of the grid attend, the others
 // score, split in proportion to their bytes (forced_ctas in
@@ -29,9 +30,8 @@ struct StreamCfg {
     static constexpr int NW = 4;                   // warps per CTA
     static constexpr int STAGES = D == 128 ? 2 : 3;  // ring stages per warp
     static constexpr int RING = STAGES * 2 * kPage * D * 2;
-    // a K+V page stage holds one bf16 metadata tile or two E4M3 tiles; the
-    // ring has an mbarrier for each of the latter
-    static constexpr int NBAR = 2 * STAGES;
+    // a K+V page stage holds one bf16 metadata tile or two E4M3 tiles
+    static constexpr int NBAR = STAGES;
     static constexpr int SMEM = NW * (RING + NBAR * 8 + STAGES * 4);
     static constexpr int MIN_BLOCKS = D == 128 ? 3 : 1;
 };
@@ -40,8 +40,7 @@ template <int D, bool FP8>
 __global__ void __launch_bounds__(StreamCfg<D>::NW * 32, StreamCfg<D>::MIN_BLOCKS)
     stream_kernel(StreamParams p) {
     using C = StreamCfg<D>;
-    static_assert(C::RING == C::STAGES * scr::TileGeom<D>::TILE_B, "ring holds NT tiles");
-    static_assert(C::RING == C::NBAR * scr::TileGeom<D, true>::TILE_B, "or 2 NT E4M3 tiles");
+    static_assert(C::RING == C::STAGES * scr::TileGeom<D>::TILE_B, "ring holds STAGES tiles");
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     Ring ring;
@@ -72,11 +71,41 @@ __global__ void __launch_bounds__(StreamCfg<D>::NW * 32, StreamCfg<D>::MIN_BLOCK
         bool ok = true;
         attend_range<D, C::NW, C::STAGES>(a, smem, ring, it, ok, s, e, blockIdx.x);
     } else if (p.sc.scores != nullptr) {
-        // candidate scores, tiles spread over the remaining CTAs' warps
-        uint32_t it = 0;
-        scr::score_range_bulk<D, FP8 ? C::NBAR : C::STAGES, FP8>(
-            p.sc, ring.tiles, ring.bars, it, (blockIdx.x - nf) * C::NW + warp,
-            (gridDim.x - nf) * C::NW);
+        // candidate scores: the tiles of all units in (b, h, tile) order, a
+        // contiguous range per warp of the remaining CTAs, each unit's
+        // segment through the warp's ring (asynchronous 16-byte copies)
+        const ScoreParams& sp = p.sc;
+        constexpr int NS = C::RING / scr::TileGeom<D, FP8>::TILE_B;
+        auto tiles_of = [&](int b) {
+            const int L = checked_len(sp.seq_lens, b, sp.max_pages, sp.status);
+            const PageRanges r = page_ranges(L, sp.prefix, sp.window);
+            return (r.ws - r.np + kSelTile - 1) / kSelTile;
+        };
+        const long long total = total_units(sp.batch, sp.hkv, tiles_of);
+        const long long nw = (long long)(gridDim.x - nf) * C::NW;
+        const long long per = (total + nw - 1) / nw;
+        long long g = ((long long)(blockIdx.x - nf) * C::NW + warp) * per;
+        const long long g_end = min(total, g + per);
+        if (g < g_end) {
+            int u;
+            long long ustart;
+            locate_unit(g, sp.batch, sp.hkv, tiles_of, &u, &ustart);
+            while (g < g_end && u < sp.batch * sp.hkv) {
+                const int L = checked_len(sp.seq_lens, u / sp.hkv, sp.max_pages, sp.status);
+                const PageRanges r = page_ranges(L, sp.prefix, sp.window);
+                const long long uend = ustart + (r.ws - r.np + kSelTile - 1) / kSelTile;
+                const long long stop = min(g_end, uend);
+                if (stop > g) {
+                    float w[scr::TileGeom<D>::CPL][8];
+                    scr::load_weights<D>(sp, u, w);
+                    scr::score_run<D, NS, FP8>(sp, ring.tiles, u, r, (int)(g - ustart),
+                                               (int)(stop - ustart), w);
+                    g = stop;
+                }
+                ustart = uend;
+                ++u;
+            }
+        }
     }
 }
 
