@@ -78,10 +78,11 @@ def page_ranges(L, prefix, window):
     return n, np_, ws
 
 
-def algorithmic_bytes(lens, hq, hkv, D, prefix, window, budget, dense=False):
-    """Bytes the step must move: metadata of candidate pages (4*D per page
-    and kv head), K and V of attended tokens (4*D per token and kv head), q
-    (bf16) and out (fp32).  Returns (total, meta, kv)."""
+def algorithmic_bytes(lens, hq, hkv, D, prefix, window, budget, dense=False, meta_bytes=2):
+    """Bytes the step must move: metadata of candidate pages (2*D*meta_bytes
+    per page and kv head: 4*D for bf16 bounds, 2*D for E4M3), K and V of
+    attended tokens (4*D per token and kv head), q (bf16) and out (fp32).
+    Returns (total, meta, kv)."""
     meta = kv = 0
     for L in lens:
         n, np_, ws = page_ranges(L, prefix, window)
@@ -89,7 +90,7 @@ def algorithmic_bytes(lens, hq, hkv, D, prefix, window, budget, dense=False):
             tokens = L
         else:
             nc = ws - np_
-            meta += nc * hkv * 4 * D
+            meta += nc * hkv * 2 * D * meta_bytes
             sel = min(budget, nc)
             tokens = min(L, 16 * np_) + 16 * sel + max(0, L - 16 * ws)
         kv += tokens * hkv * 4 * D
@@ -211,7 +212,7 @@ def ncu_traffic():
 class Workload:
     """Device-resident inputs of one workload (single layer)."""
 
-    def __init__(self, name, extra_tokens=0, copies=1):
+    def __init__(self, name, extra_tokens=0, copies=1, meta_format="bf16"):
         import torch
         import sparse_long_context_max_b200 as slc
         import synth
@@ -225,7 +226,7 @@ class Workload:
         # steps can run on different layers, as a model's do
         self.caches = []
         for _ in range(copies):
-            c = slc.PagedCache(x.k_cache.cuda(), x.v_cache.cuda())
+            c = slc.PagedCache(x.k_cache.cuda(), x.v_cache.cuda(), meta_format=meta_format)
             slc.build_page_meta(c, self.bt, self.sl)
             self.caches.append(c)
         self.cache = self.caches[0]
@@ -591,6 +592,24 @@ def run_ours(args, rank, world, local):
                   "decode256k_dense_gbs": round(db256 / (dn * 1e-3) / 1e9, 1)}
         assert slc.device_status() == 0
         del gsp, gdn, W256
+        torch.cuda.empty_cache()
+        # the same step over E4M3 page bounds (outward-rounded): half the
+        # metadata bytes
+        W8 = Workload("decode256k", meta_format="fp8")
+        b8 = algorithmic_bytes(lens256, y.wl.hq, y.wl.hkv, y.wl.head_dim, y.prefix, y.window,
+                               y.budget, meta_bytes=1)
+        g8 = graph_of(lambda: slc.sparse_decode(W8.q, W8.cache, W8.bt, W8.sl, y.prefix,
+                                                y.window, y.budget, out=W8.out,
+                                                workspace=W8.ws))
+        sp8 = timed(g8.replay, max(reps, 32), None)
+        gbs8 = b8[0] / (sp8 * 1e-3) / 1e9
+        top256.update({"decode256k_fp8meta_sparse_us": round(sp8 * 1e3, 2),
+                       "decode256k_fp8meta_speedup_vs_dense": round(dn / sp8, 2),
+                       "decode256k_fp8meta_hbm_gbs": round(gbs8, 1),
+                       "decode256k_fp8meta_roofline_frac": round(gbs8 / peak, 4),
+                       "decode256k_fp8meta_algorithmic_bytes": b8[0]})
+        assert slc.device_status() == 0
+        del g8, W8
         torch.cuda.empty_cache()
         if not args.no_also:
             for name in ("tiny", "ragged"):

@@ -57,3 +57,10 @@ def test_dense_bytes_are_every_token():
     assert m == 0
     assert k == sum(lens) * 2 * 4 * 32
     assert np.isclose(total, k + 3 * 8 * 32 * 6)
+
+
+def test_e4m3_metadata_halves_the_metadata_bytes():
+    lens = [1000, 333, 130]
+    t2, m2, k2 = bench.algorithmic_bytes(lens, 8, 2, 32, 40, 100, 5)
+    t1, m1, k1 = bench.algorithmic_bytes(lens, 8, 2, 32, 40, 100, 5, meta_bytes=1)
+    assert m1 * 2 == m2 and k1 == k2 and t2 - t1 == m1
