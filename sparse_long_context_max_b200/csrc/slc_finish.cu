@@ -46,18 +46,19 @@ namespace {
 namespace cg = cooperative_groups;
 using namespace attn;
 
-// Four warps, all attending: the attention needs ~150 (d = 128) to ~250
-// (d = 256) registers per thread, and two CTAs must fit on an SM so that one
-// cluster per unit is co-resident for the usual unit counts.  (Eight warps
-// of 128 registers with one ring stage each measured slower.)
+// Eight warps, all attending, one CTA per SM: a unit's clusters take at
+// most one CTA per SM anyway at the usual unit counts, and with two warps
+// per scheduler the latency-bound per-page work of the attention and the
+// selection's steps overlap (four warps per CTA, two CTAs per SM, left one
+// warp per scheduler busy and measured slower).
 template <int D>
 struct FinishCfg {
-    static constexpr int NT = 128;                     // threads per CTA
+    static constexpr int NT = 256;                     // threads per CTA
     static constexpr int NW = NT / 32;                 // warps per CTA
     static constexpr int NW_ATT = NW;                  // warps that attend
     static constexpr int STAGES = D == 128 ? 2 : 1;    // ring stages per attending warp
     static constexpr int RING = STAGES * 2 * kPage * D * 2;
-    static constexpr int MIN_BLOCKS = 2;
+    static constexpr int MIN_BLOCKS = 1;
 };
 
 constexpr int kBins = 256;       // 8-bit digits
@@ -162,6 +163,40 @@ __device__ __forceinline__ void scan_digit(const FinishShared& sh, int remaining
     *digit = __shfl_sync(0xffffffffu, d, src);
     *above = __shfl_sync(0xffffffffu, ab, src);
     *count = __shfl_sync(0xffffffffu, ct, src);
+}
+
+// The k-th largest of the keys one warp holds in registers (NK per lane,
+// only the first nk used; key 0: none), 1 <= k <= their count, by
+// bit-by-bit bisection from the highest bit where the warp's smallest and
+// largest keys differ: each bit, every lane counts its keys >= T | bit and
+// one warp reduction sums the counts (no barrier).  With max_bits below the
+// bits left the result is a lower bound (at least k keys are >= it).
+template <int NK>
+__device__ __forceinline__ uint32_t warp_kth(const uint32_t (&v)[NK], int nk, int k,
+                                             int max_bits) {
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+    for (int c = 0; c < NK; ++c)
+        if (c < nk && v[c]) {
+            kmin = min(kmin, v[c]);
+            kmax = max(kmax, v[c]);
+        }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (kmin >= kmax) return kmin;
+    const int hb = 31 - __clz(kmin ^ kmax);
+    uint32_t T = hb == 31 ? 0u : kmin & ~((2u << hb) - 1u);
+    const int lo = max(0, hb + 1 - max_bits);
+    for (int bit = hb; bit >= lo; --bit) {
+        const uint32_t tr = T | (1u << bit);
+        int part[4] = {0, 0, 0, 0};  // four partial sums: a shorter add chain
+#pragma unroll
+        for (int c = 0; c < NK; ++c)
+            if (c < nk) part[c & 3] += v[c] >= tr ? 1 : 0;
+        const int cnt = __reduce_add_sync(0xffffffffu, (part[0] + part[1]) + (part[2] + part[3]));
+        if (cnt >= k) T = tr;
+    }
+    return T;
 }
 
 // The cluster-wide k-th largest key: the k largest keys of the unit are the
@@ -488,10 +523,31 @@ __global__ void __launch_bounds__(FinishCfg<D>::NT, FinishCfg<D>::MIN_BLOCKS)
             __syncthreads();
             bool fast = false;
             if (bound) {
-                uint32_t tT;
-                int tties;
-                cta_kth<NT>(tkeys, 1, ntiles, nsel, sh, &tT, &tties);
-                const uint32_t tau = tties > 0 ? tT : tT + 1u;  // the nsel-th largest maximum
+                // tau: each warp's ceil(nsel / NW)-th largest tile maximum
+                // among its share of the tiles (ballot-free bisection, ten
+                // bits: a lower bound), the smallest over the warps; at least
+                // nsel tile maxima (distinct keys) are >= it whenever every
+                // warp holds that many, else tau = 0 (every key survives)
+                uint32_t tau;
+                {
+                    constexpr int TC = kMaxCandidates / kSelTile / NT;  // tile keys per lane
+                    const int kw = (nsel + NW - 1) / NW;
+                    const int tspan = (ntiles + NW - 1) / NW;
+                    const int t0 = warp * tspan, t1 = min(ntiles, t0 + tspan);
+                    uint32_t v[TC];
+#pragma unroll
+                    for (int c = 0; c < TC; ++c) {
+                        const int t = t0 + 32 * c + lane;
+                        v[c] = t < t1 ? tkeys[t] : 0u;
+                    }
+                    const bool enough = t1 - t0 >= kw;
+                    const uint32_t vw = enough ? warp_kth<TC>(v, (tspan + 31) / 32, kw, 10) : 0u;
+                    if (lane == 0) sh.red_min[warp] = vw;
+                    __syncthreads();
+                    tau = 0xffffffffu;
+#pragma unroll
+                    for (int w2 = 0; w2 < NW; ++w2) tau = min(tau, sh.red_min[w2]);
+                }
                 cp_async_wait<0>();  // this thread's phys[] copies
                 __syncthreads();     // every phys[] copy landed; tkeys is no longer read
                 // this CTA's survivors, in index order, over the tile maxima
@@ -514,19 +570,7 @@ __global__ void __launch_bounds__(FinishCfg<D>::NT, FinishCfg<D>::MIN_BLOCKS)
                     const bool keep = i < w1 && keys[i] >= tau;
                     const unsigned bk = __ballot_sync(0xffffffffu, keep);
                     const int pos = before + __popc(bk & below);
-                    if (keep && pos < kOwnSurvivorCap) {
-                        const int ph = phys[i];
-                        own[pos] = Survivor{keys[i], c0 + i, ph, 0};
-                        // every selected page is a survivor: its K and V start
-                        // their way into L2 now, while HBM idles through the
-                        // rest of the selection
-                        if (ph >= 0 && ph < a.num_pages) {
-                            constexpr uint32_t TILE = kPage * D * 2;
-                            const long long off = ((long long)ph * a.hkv + h) * TILE;
-                            prefetch_l2(static_cast<const uint8_t*>(a.k_cache) + off, TILE);
-                            prefetch_l2(static_cast<const uint8_t*>(a.v_cache) + off, TILE);
-                        }
-                    }
+                    if (keep && pos < kOwnSurvivorCap) own[pos] = Survivor{keys[i], c0 + i, phys[i], 0};
                     before += __popc(bk);
                 }
                 if (tid == 0) sh.scount = nown;
@@ -773,9 +817,11 @@ cudaError_t setup_one(DeviceCfg& d, int di) {
     for (int ci = 0; ci < kNumFinishClusters; ++ci) {
         const int c = kFinishClusters[ci];
         const size_t smem = finish_smem<D>(c);
-        cudaError_t e = cudaFuncSetAttribute(finish_kernel<D>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)finish_smem<D>(8));
+        // the smallest cluster needs the most shared memory (the largest
+        // slices of the candidates)
+        cudaError_t e = cudaFuncSetAttribute(
+            finish_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            (int)finish_smem<D>(kFinishClusters[kNumFinishClusters - 1]));
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(finish_kernel<D>,
                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
