@@ -156,18 +156,22 @@ __device__ void warp_attend(const AttendParams& p, const Ring& ring, uint32_t& i
                 reinterpret_cast<const uint32_t*>(ring.tiles) + stage * 2 * TILE_W;
             const uint32_t* Vw = Kw + TILE_W;
 
-            // S = Q K^T for tokens nb*8 + (0..7)
+            // S = Q K^T for tokens nb*8 + (0..7): two accumulators per block
+            // (even and odd k-steps) halve the dependent chain of mma
             float s[2][4];
 #pragma unroll
             for (int nb = 0; nb < 2; ++nb) {
+                float s2[4] = {0.f, 0.f, 0.f, 0.f};
                 s[nb][0] = s[nb][1] = s[nb][2] = s[nb][3] = 0.f;
                 const uint32_t* krow = Kw + (nb * 8 + r_) * ROW_W;
 #pragma unroll
                 for (int m = 0; m < D / 32; ++m) {
                     const uint4 kv = lds128(krow + (c_ + 4 * m) * 4);
                     mma_bf16(s[nb], qa[2 * m][0], 0u, qa[2 * m][1], 0u, kv.x, kv.y);
-                    mma_bf16(s[nb], qa[2 * m + 1][0], 0u, qa[2 * m + 1][1], 0u, kv.z, kv.w);
+                    mma_bf16(s2, qa[2 * m + 1][0], 0u, qa[2 * m + 1][1], 0u, kv.z, kv.w);
                 }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) s[nb][e] += s2[e];
             }
             // this thread: head r_, tokens 2c, 2c+1, 8+2c, 9+2c
             const int t0 = 2 * c_;
@@ -378,9 +382,10 @@ __device__ __forceinline__ long long unit_list_start(const AttendParams& p, int 
 // The streaming kernel's split of its grid (slc_stream.cu): the first
 // forced_ctas(...) CTAs attend the prefix/window lists (one chunk each), the
 // others score the candidate tiles, so the two run side by side.  A forced
-// page (K + V) and a 16-page metadata tile are both 64*D bytes, so the CTAs
-// are split in proportion to the counts, with at least one CTA for a
-// non-empty side and at least kMinForcedPages pages per attending CTA.
+// page (K + V) and a 16-page bf16 metadata tile are both 64*D bytes; the
+// CTAs are split so that both sides end together (a tile costs a CTA about
+// 1.5 pages' time), with at least one CTA for a non-empty side and at least
+// kMinForcedPages pages per attending CTA.
 // Warp-wide (every lane gets the result); the finishing
 // kernel recomputes it to find the prefix/window partials.
 constexpr int kMinForcedPages = 8;
@@ -392,13 +397,16 @@ __device__ __forceinline__ int forced_ctas(const AttendParams& a, bool scoring, 
         const PageRanges r = page_ranges(L, a.prefix, a.window);
         return (r.ws - r.np + kSelTile - 1) / kSelTile;
     };
-    const long long f = total_units(a.batch, a.hkv, forced_of);
-    const long long t = scoring ? total_units(a.batch, a.hkv, tiles_of) : 0;
+    // a CTA attends about 1.5x the bytes per unit time that it scores
+    // (measured at 64k and 256k), so a tile weighs 3 and a page 2
+    const long long pages = total_units(a.batch, a.hkv, forced_of);
+    const long long f = 2 * pages;
+    const long long t = scoring ? 3 * total_units(a.batch, a.hkv, tiles_of) : 0;
     if (f == 0) return t == 0 ? grid : 0;
     long long n = t == 0 ? grid : (f * grid + (f + t) / 2) / (f + t);
     // at least kMinForcedPages pages per attending CTA: fewer, fuller chunks
     // (each chunk of a unit's list is one partial for the finishing kernel)
-    n = min(n, (f + kMinForcedPages - 1) / kMinForcedPages);
+    n = min(n, (pages + kMinForcedPages - 1) / kMinForcedPages);
     if (n < 1) n = 1;
     if (t > 0 && n > grid - 1) n = grid - 1;
     return (int)n;
