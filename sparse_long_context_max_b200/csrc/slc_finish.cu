@@ -100,12 +100,13 @@ struct FinishLayout {
     static constexpr size_t bars = (size_t)C::NW_ATT * C::RING;
     static constexpr size_t nvalid = bars + C::NW_ATT * C::STAGES * 8;
     static constexpr size_t keys = (nvalid + C::NW_ATT * C::STAGES * 4 + 127) / 128 * 128;
-    static constexpr size_t phys(int cluster) {
-        return keys + (size_t)(kMaxCandidates / cluster) * 4;
+    // a CTA's slice of the candidates, at most (rounded up to 4 keys, as
+    // the kernel rounds its slices)
+    static constexpr size_t slice(int cluster) {
+        return (size_t)(((kMaxCandidates + cluster - 1) / cluster + 3) / 4 * 4);
     }
-    static constexpr size_t shared(int cluster) {
-        return phys(cluster) + (size_t)(kMaxCandidates / cluster) * 4;
-    }
+    static constexpr size_t phys(int cluster) { return keys + slice(cluster) * 4; }
+    static constexpr size_t shared(int cluster) { return phys(cluster) + slice(cluster) * 4; }
     static constexpr size_t part(int cluster) { return shared(cluster) + sizeof(FinishShared); }
     static constexpr size_t total(int cluster) {
         return part(cluster) + (kMaxGroup * D + 2 * kMaxGroup) * 4;
