@@ -51,6 +51,9 @@ def _load(path=None):
             lib.oracle_page_scores.restype = None
             lib.oracle_select_pages.argtypes = [P, I, I, P, I, I, I, I, P, P]
             lib.oracle_select_pages.restype = None
+            lib.oracle_select_pages_delta.argtypes = [P, I, I, P, I, I, I, I,
+                                                      ctypes.c_double, I, P, P]
+            lib.oracle_select_pages_delta.restype = None
             lib.oracle_attend.argtypes = [P, P, P, I, I, I, I, P, I, P, I, I, I,
                                           P, I, I, ctypes.c_double, P]
             lib.oracle_attend.restype = I
@@ -201,6 +204,23 @@ def select_pages(scores, seq_lens, prefix: int, window: int, budget: int):
     lib.oracle_select_pages(_ptr(s), hkv, max_pages, _ptr(sl), B, int(prefix),
                             int(window), int(budget), _ptr(sel), _ptr(nsel))
     return sel, nsel
+
+
+def select_pages_delta(scores, seq_lens, prefix: int, window: int, d: int, delta: float,
+                       cap: int):
+    """Top-delta selection per (b, kv head): the d best candidates plus every
+    candidate within delta of the best, ascending, -1 padded to cap (the cap
+    best of the union if it is larger): (sel [B][Hkv][cap], nsel [B][Hkv])."""
+    lib = _load()
+    s = np.ascontiguousarray(scores, dtype=np.float64)
+    B, hkv, max_pages = s.shape
+    sl = _i32(seq_lens)
+    sel = np.empty((B, hkv, max(cap, 1)), dtype=np.int32)
+    nsel = np.empty((B, hkv), dtype=np.int32)
+    lib.oracle_select_pages_delta(_ptr(s), hkv, max_pages, _ptr(sl), B, int(prefix),
+                                  int(window), int(d), float(delta), int(cap), _ptr(sel),
+                                  _ptr(nsel))
+    return sel[:, :, :cap], nsel
 
 
 def attend(q, k_cache, v_cache, block_table, seq_lens, prefix: int = 0,

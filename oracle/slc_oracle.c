@@ -329,6 +329,57 @@ void oracle_select_pages(const double *scores, int hkv, int max_pages,
     free(keep);
 }
 
+/* Top-delta selection ("Faster Than Flash: Fudan FFD Hits 11.6x Kernel
+ * Speedup, Pushes Long-Context Decoding to 256K", section "top-delta: Tearing
+ * Down "Global Synchronization" Too"): per (sequence, kv head), the d
+ * candidate pages with the highest scores (the order of oracle_select_pages)
+ * together with every candidate page whose score is within delta of the
+ * highest candidate score (s_max - s_j <= delta).  Readings: d and delta are
+ * given per call; the union is written in ascending page order, -1 padded to
+ * cap, and if it holds more than cap pages the cap best of it (score desc,
+ * page asc) are kept.  nsel receives the count written. */
+void oracle_select_pages_delta(const double *scores, int hkv, int max_pages,
+                               const int32_t *seq_lens, int batch, int prefix,
+                               int window, int d, double delta, int cap,
+                               int32_t *sel, int32_t *nsel)
+{
+    ranked_t *buf = (ranked_t *)malloc(sizeof(ranked_t) * (max_pages > 0 ? max_pages : 1));
+    int *keep = (int *)malloc(sizeof(int) * (max_pages > 0 ? max_pages : 1));
+    for (int b = 0; b < batch; b++) {
+        int n, np, ws;
+        oracle_page_ranges(seq_lens[b], prefix, window, &n, &np, &ws);
+        for (int h = 0; h < hkv; h++) {
+            const double *s = scores + ((int64_t)b * hkv + h) * max_pages;
+            int m = 0;
+            double smax = -INFINITY;
+            for (int j = np; j < ws; j++) {
+                buf[m].score = s[j];
+                buf[m].page = j;
+                if (s[j] > smax)
+                    smax = s[j];
+                m++;
+            }
+            qsort(buf, m, sizeof(ranked_t), rank_cmp);
+            /* the union, in rank order: the first d ranked pages, and every
+             * page within delta of the top */
+            int k = 0;
+            for (int i = 0; i < m; i++) {
+                const int in_top = i < d;
+                const int near = smax - buf[i].score <= delta;
+                if ((in_top || near) && k < cap)
+                    keep[k++] = buf[i].page;
+            }
+            qsort(keep, k, sizeof(int), int_cmp);
+            int32_t *out = sel + ((int64_t)b * hkv + h) * cap;
+            for (int i = 0; i < cap; i++)
+                out[i] = i < k ? keep[i] : -1;
+            nsel[b * hkv + h] = k;
+        }
+    }
+    free(buf);
+    free(keep);
+}
+
 /* Softmax attention of one query head over an explicit token list. */
 static void attend_tokens(const uint16_t *qh, const uint16_t *k_cache,
                           const uint16_t *v_cache, int hkv, int h, int dim,

@@ -420,3 +420,62 @@ def test_fp8_bounds_of_a_page_grow_one_token_at_a_time():
                 hi = max(oracle.fp8_value(a8[1][0, h, 0, d]), oracle.fp8_value(up))
                 assert oracle.fp8_value(b8[0][0, h, 0, d]) == lo
                 assert oracle.fp8_value(b8[1][0, h, 0, d]) == hi
+
+
+# ------------------------------------------------------------------ top-delta
+
+def _delta_scores(fx):
+    n = -(-fx["length"] // 16)
+    s = np.full((1, 1, n), np.nan)
+    s[0, 0, :] = fx["scores"]
+    return s
+
+
+def test_top_delta_golden():
+    fx = json.load(open(os.path.join(GOLDEN, "top_delta.json")))
+    s = _delta_scores(fx)
+    for c in fx["cases"]:
+        sel, nsel = oracle.select_pages_delta(s, [fx["length"]], fx["prefix"], fx["window"],
+                                              c["d"], c["delta"], c["cap"])
+        want = c["selected"] + [-1] * (c["cap"] - len(c["selected"]))
+        assert sel[0, 0].tolist() == want, c
+        assert int(nsel[0, 0]) == len(c["selected"]), c
+
+
+def test_top_delta_is_a_longer_top_k():
+    """The top d and the pages within delta of the best are both prefixes of
+    the (score desc, page asc) order, so their union is the top k with
+    k = max(d, #within delta), capped: the plain selection with that budget."""
+    rng = np.random.default_rng(5)
+    for trial in range(40):
+        B, hkv, mp = 2, 2, 90
+        lens = rng.integers(1, mp * 16, size=B).astype(np.int32)
+        prefix, window = int(rng.integers(0, 60)), int(rng.integers(0, 300))
+        s = np.round(rng.normal(size=(B, hkv, mp)) * 4) / 4  # many exact ties
+        d = int(rng.integers(0, 12))
+        delta = float(rng.choice([0.0, 0.25, 0.5, 1.0, 2.5]))
+        cap = int(rng.integers(1, 40))
+        sel, nsel = oracle.select_pages_delta(s, lens, prefix, window, d, delta, cap)
+        for b in range(B):
+            n, np_, ws = oracle.page_ranges(int(lens[b]), prefix, window)
+            for h in range(hkv):
+                cand = s[b, h, np_:ws]
+                m = int((cand.max() - cand <= delta).sum()) if cand.size else 0
+                k = min(max(d, m), cap, cand.size)
+                ref, rn = oracle.select_pages(s[b:b + 1, h:h + 1], lens[b:b + 1], prefix, window, k)
+                assert int(nsel[b, h]) == k == int(rn[0, 0])
+                assert sel[b, h, :k].tolist() == ref[0, 0, :k].tolist()
+                assert (sel[b, h, k:] == -1).all()
+
+
+def test_top_delta_edges():
+    rng = np.random.default_rng(6)
+    s = rng.normal(size=(1, 2, 50))
+    lens = [800]
+    top, _ = oracle.select_pages(s, lens, 16, 64, 7)
+    neg, nn = oracle.select_pages_delta(s, lens, 16, 64, 7, -1.0, 7)
+    assert (neg == top).all() and (nn == 7).all()  # a negative delta adds nothing
+    n, np_, ws = oracle.page_ranges(800, 16, 64)
+    allc, na = oracle.select_pages_delta(s, lens, 16, 64, 0, np.inf, 60)
+    assert (na == ws - np_).all()  # an infinite delta keeps every candidate
+    assert allc[0, 0, : ws - np_].tolist() == list(range(np_, ws))

@@ -43,6 +43,11 @@ MUTANTS = [
      "kmax8[base + d] = (uint8_t)oracle_fp8_round(kmax[base + d], kmax[base + d] - oracle_fp8_value(oracle_fp8_round(kmax[base + d], 0)) > oracle_fp8_value(oracle_fp8_round(kmax[base + d], 1)) - kmax[base + d]);"),
     ("fp8 rounding off by one code", "return lo < fp8_count ? fp8_table[lo].code : 0x7F;",
      "return lo + 1 < fp8_count ? fp8_table[lo + 1].code : 0x7F;"),
+    ("top-delta gap strict", "const int near = smax - buf[i].score <= delta;",
+     "const int near = smax - buf[i].score < delta;"),
+    ("top-delta one page short of d", "const int in_top = i < d;", "const int in_top = i < d - 1;"),
+    ("top-delta cap keeps the lowest pages", "if ((in_top || near) && k < cap)",
+     "if (in_top || near)"),
 ]
 
 
