@@ -165,6 +165,23 @@ SLC_API int slc_select_pages(const float *scores, int32_t num_kv_heads, int32_t 
                      const int32_t *seq_lens, int32_t batch, int32_t prefix, int32_t window,
                      int32_t budget, int32_t *selected, slc_stream_t stream);
 
+/* Top-delta selection ("Faster Than Flash: Fudan FFD Hits 11.6x Kernel
+ * Speedup, Pushes Long-Context Decoding to 256K", section "top-delta: Tearing
+ * Down "Global Synchronization" Too"): per (sequence, kv head), the d
+ * candidate pages with the highest scores together with every candidate
+ * page whose score is within delta of the highest candidate score
+ * (s_max - s_j <= delta, the threshold computed in fp32), at most cap pages
+ * (the cap best of that union, best = higher score, then lower page).
+ * Scores as slc_score_pages writes them.  selected: int32
+ * [batch][num_kv_heads][cap], ascending page indices, padded with -1.
+ * d >= 0, cap >= 0, delta not NaN (+inf keeps every candidate, a negative
+ * delta only the top d); SLC_ERR_INVALID_ARG otherwise.  Candidate counts
+ * up to 32768 pages. */
+SLC_API int slc_select_pages_delta(const float *scores, int32_t num_kv_heads,
+                           int32_t max_pages_per_seq, const int32_t *seq_lens, int32_t batch,
+                           int32_t prefix, int32_t window, int32_t d, float delta, int32_t cap,
+                           int32_t *selected, slc_stream_t stream);
+
 /* One decode step of one layer, in two kernels:
  *   1 (streaming)  attention over the prefix and window pages, and the
  *                  scores of the candidate pages (all SMs, HBM-bound);
@@ -213,6 +230,20 @@ SLC_API int slc_sparse_attend(const void *q, const slc_cache_t *cache, const int
                       int32_t num_q_heads, int32_t prefix, int32_t window, int32_t budget,
                       const int32_t *selected, float scale, float *out, void *workspace,
                       size_t workspace_bytes, slc_stream_t stream);
+
+/* One decode step with the top-delta selection in place of the fixed
+ * budget: the candidate scores (slc_score_pages), the top-delta selection
+ * (slc_select_pages_delta, into selected_out when given, else the
+ * workspace), then attention over the prefix, window and selected pages and
+ * the merge (as slc_sparse_attend): four kernels.  workspace >=
+ * slc_workspace_size(..., budget = cap).  Other arguments as
+ * slc_sparse_decode and slc_select_pages_delta. */
+SLC_API int slc_sparse_decode_delta(const void *q, const slc_cache_t *cache,
+                            const int32_t *block_table, int32_t max_pages_per_seq,
+                            const int32_t *seq_lens, int32_t batch, int32_t num_q_heads,
+                            int32_t prefix, int32_t window, int32_t d, float delta,
+                            int32_t cap, float scale, float *out, int32_t *selected_out,
+                            void *workspace, size_t workspace_bytes, slc_stream_t stream);
 
 /* Full attention over every token of every sequence (the comparison
  * point: a full-attention layer reads every key at each step, "Hybrid LLM

@@ -24,7 +24,8 @@ from . import _build
 
 __all__ = [
     "SLCError", "PagedCache", "kv_append", "build_page_meta", "workspace_size",
-    "score_pages", "select_pages", "sparse_decode", "sparse_attend", "dense_decode",
+    "score_pages", "select_pages", "select_pages_delta", "sparse_decode", "sparse_decode_delta",
+    "sparse_attend", "dense_decode",
     "device_status",
     "library_path", "KERNELS_PER_CALL", "STATUS_BITS", "META_FORMATS",
 ]
@@ -35,7 +36,8 @@ PAGE = 16
 # kernel, then the finishing kernel; dense: attend, merge)
 KERNELS_PER_CALL = {"sparse_decode": 2, "sparse_decode_stage": 1, "dense_decode": 2,
                     "sparse_attend": 2, "kv_append": 1,
-                    "build_page_meta": 1, "score_pages": 1, "select_pages": 1}
+                    "build_page_meta": 1, "score_pages": 1, "select_pages": 1,
+                    "select_pages_delta": 1, "sparse_decode_delta": 4}
 
 STATUS_BITS = {1: "bad page", 2: "bad length", 4: "bad selection", 8: "wait timeout"}
 
@@ -70,6 +72,8 @@ def _load() -> ctypes.CDLL:
         "slc_workspace_size": (Z, [I, I, I, I, I, I]),
         "slc_score_pages": (I, [P, C, P, I, P, I, I, I, I, P, P]),
         "slc_select_pages": (I, [P, I, I, P, I, I, I, I, P, P]),
+        "slc_select_pages_delta": (I, [P, I, I, P, I, I, I, I, F, I, P, P]),
+        "slc_sparse_decode_delta": (I, [P, C, P, I, P, I, I, I, I, I, F, I, F, P, P, P, Z, P]),
         "slc_sparse_decode": (I, [P, C, P, I, P, I, I, I, I, I, F, P, P, P, Z, P]),
         "slc_dense_decode": (I, [P, C, P, I, P, I, I, F, P, P, Z, P]),
         "slc_sparse_attend": (I, [P, C, P, I, P, I, I, I, I, I, P, F, P, P, Z, P]),
@@ -205,6 +209,20 @@ def select_pages(scores, seq_lens, prefix, window, budget, selected=None):
     return selected
 
 
+def select_pages_delta(scores, seq_lens, prefix, window, d, delta, cap, selected=None):
+    """Top-delta selection: per (b, kv head) the d best candidate pages plus
+    every candidate within delta of the best, at most cap; int32
+    [B][Hkv][cap] ascending, -1 padded."""
+    _need(scores, torch.float32, "scores", 3)
+    B, hkv, mp = scores.shape
+    if selected is None:
+        selected = torch.empty((B, hkv, cap), dtype=torch.int32, device=scores.device)
+    _check(_lib.slc_select_pages_delta(_ptr(scores), hkv, mp, _ptr(seq_lens), B, prefix, window,
+                                       int(d), float(delta), int(cap), _ptr(selected),
+                                       _stream()))
+    return selected
+
+
 _ws_cache: dict = {}
 
 
@@ -236,6 +254,31 @@ def sparse_decode(q, cache: PagedCache, block_table, seq_lens, prefix, window, b
                                   hq, prefix, window, budget, float(scale), _ptr(out),
                                   _ptr(selected_out), _ptr(workspace), workspace.numel(),
                                   _stream()))
+    return out
+
+
+def sparse_decode_delta(q, cache: PagedCache, block_table, seq_lens, prefix, window, d, delta,
+                        cap, scale=0.0, out=None, selected_out=None, workspace=None):
+    """One decode step with the top-delta selection (the d best candidate
+    pages plus every candidate within delta of the best, at most cap) in
+    place of the fixed budget; returns out (fp32 [B][Hq][D])."""
+    _need(q, torch.bfloat16, "q", 3)
+    _need(block_table, torch.int32, "block_table", 2)
+    _need(seq_lens, torch.int32, "seq_lens", 1)
+    B, hq, dim = q.shape
+    mp = block_table.shape[1]
+    if out is None:
+        out = torch.empty((B, hq, dim), dtype=torch.float32, device=q.device)
+    _need(out, torch.float32, "out", 3)
+    if selected_out is not None:
+        _need(selected_out, torch.int32, "selected_out", 3)
+    need = workspace_size(B, hq, cache.num_kv_heads, dim, mp, cap)
+    if workspace is None:
+        workspace = _workspace(q.device, need)
+    _check(_lib.slc_sparse_decode_delta(_ptr(q), cache.c, _ptr(block_table), mp, _ptr(seq_lens),
+                                        B, hq, prefix, window, int(d), float(delta), int(cap),
+                                        float(scale), _ptr(out), _ptr(selected_out),
+                                        _ptr(workspace), workspace.numel(), _stream()))
     return out
 
 

@@ -214,7 +214,26 @@ int slc_select_pages(const float* scores, int32_t num_kv_heads, int32_t max_page
     int rc;
     if ((rc = device_cfg(&dev))) return rc;
     SelectParams p{scores, seq_lens, selected, dev->status, batch, num_kv_heads,
-                   max_pages_per_seq, prefix, window, budget, 0};
+                   max_pages_per_seq, prefix, window, budget, 0, -1, 0.f};
+    cudaError_t e = launch_select(p, stream);
+    return e == cudaSuccess ? SLC_OK : note_cuda(e);
+}
+
+int slc_select_pages_delta(const float* scores, int32_t num_kv_heads, int32_t max_pages_per_seq,
+                           const int32_t* seq_lens, int32_t batch, int32_t prefix,
+                           int32_t window, int32_t d, float delta, int32_t cap,
+                           int32_t* selected, slc_stream_t stream) {
+    if (batch < 0 || num_kv_heads <= 0 || max_pages_per_seq <= 0 || prefix < 0 ||
+        window < 0 || d < 0 || cap < 0 || delta != delta)
+        return SLC_ERR_INVALID_ARG;
+    if (max_pages_per_seq > kMaxCandidates) return SLC_ERR_UNSUPPORTED;
+    if (batch == 0 || cap == 0) return SLC_OK;
+    if (!scores || !seq_lens || !selected) return SLC_ERR_INVALID_ARG;
+    const DeviceCfg* dev;
+    int rc;
+    if ((rc = device_cfg(&dev))) return rc;
+    SelectParams p{scores, seq_lens, selected, dev->status, batch, num_kv_heads,
+                   max_pages_per_seq, prefix, window, cap, 0, d, delta};
     cudaError_t e = launch_select(p, stream);
     return e == cudaSuccess ? SLC_OK : note_cuda(e);
 }
@@ -358,6 +377,38 @@ int slc_sparse_attend(const void* q, const slc_cache_t* cache, const int32_t* bl
     return decode(2, q, cache, block_table, max_pages_per_seq, seq_lens, batch, num_q_heads,
                   prefix, window, budget, scale, out, const_cast<int32_t*>(selected), workspace,
                   workspace_bytes, stream);
+}
+
+int slc_sparse_decode_delta(const void* q, const slc_cache_t* cache, const int32_t* block_table,
+                            int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                            int32_t num_q_heads, int32_t prefix, int32_t window, int32_t d,
+                            float delta, int32_t cap, float scale, float* out,
+                            int32_t* selected_out, void* workspace, size_t workspace_bytes,
+                            slc_stream_t stream) {
+    bool empty;
+    int rc = check_decode(1, q, cache, block_table, max_pages_per_seq, seq_lens, batch,
+                          num_q_heads, prefix, window, cap, scale, out, selected_out, &empty);
+    if (rc) return rc;
+    if (d < 0 || delta != delta) return SLC_ERR_INVALID_ARG;
+    if (empty) return SLC_OK;
+    if (!workspace || !aligned16(workspace)) return SLC_ERR_INVALID_ARG;
+    const int hkv = cache->num_kv_heads;
+    const WorkspaceLayout w =
+        workspace_layout(batch, num_q_heads, hkv, cache->head_dim, max_pages_per_seq, cap);
+    if (workspace_bytes < w.total) return SLC_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    // scores by page in the scores region (rows of max_pages floats fit its
+    // rows of cand_stride), the selection in selected_out or the workspace
+    float* scores = reinterpret_cast<float*>(ws + w.scores);
+    int32_t* sel = selected_out ? selected_out : reinterpret_cast<int32_t*>(ws + w.selected);
+    rc = slc_score_pages(q, cache, block_table, max_pages_per_seq, seq_lens, batch, num_q_heads,
+                         prefix, window, scores, stream);
+    if (rc) return rc;
+    rc = slc_select_pages_delta(scores, hkv, max_pages_per_seq, seq_lens, batch, prefix, window,
+                                d, delta, cap, sel, stream);
+    if (rc) return rc;
+    return decode(2, q, cache, block_table, max_pages_per_seq, seq_lens, batch, num_q_heads,
+                  prefix, window, cap, scale, out, sel, workspace, workspace_bytes, stream);
 }
 
 int slc_dense_decode(const void* q, const slc_cache_t* cache, const int32_t* block_table,

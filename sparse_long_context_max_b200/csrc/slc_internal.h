@@ -109,6 +109,10 @@ struct SelectParams {
     unsigned* status;
     int batch, hkv, max_pages, prefix, window, budget;
     int cand_stride;
+    // top-delta when topd >= 0: the topd best candidates plus every candidate
+    // within delta of the best, at most budget; else the budget best
+    int topd;
+    float delta;
 };
 
 // Candidates per scoring tile, and the row stride of candidate-indexed

@@ -275,16 +275,13 @@ __device__ void select_unit(const SelectParams& p, int u, Scratch<NTHR>& sc, uin
     const int L = checked_len(p.seq_lens, b, p.max_pages, p.status);
     const PageRanges r = page_ranges(L, p.prefix, p.window);
     const int ncand = r.ws - r.np;
-    const int nsel = min(p.budget, ncand);
+    const bool delta_mode = p.topd >= 0;  // nsel is then decided from the scores
+    int nsel = min(p.budget, ncand);
     int32_t* out = p.selected + (long long)u * p.budget;
 
-    if (nsel >= ncand) {  // every candidate is kept (also covers ncand == 0)
-        for (int i = tid; i < p.budget; i += NTHR) out[i] = i < ncand ? r.np + i : -1;
-        if (bulk) (void)landed();
-        return;
-    }
-    for (int i = nsel + tid; i < p.budget; i += NTHR) out[i] = -1;
-    if (nsel <= 0) {
+    if ((!delta_mode && nsel >= ncand) || nsel <= 0) {
+        // every candidate is kept (or none: no candidate, or budget 0)
+        for (int i = tid; i < p.budget; i += NTHR) out[i] = i < nsel ? r.np + i : -1;
         if (bulk) (void)landed();
         return;
     }
@@ -319,6 +316,36 @@ __device__ void select_unit(const SelectParams& p, int u, Scratch<NTHR>& sc, uin
         key[k] = k < n_t ? order_key(f[k]) : 0u;
         kmax = max(kmax, key[k]);
     }
+    if (delta_mode) {
+        // top-delta ("Faster Than Flash: Fudan FFD Hits 11.6x Kernel Speedup,
+        // Pushes Long-Context Decoding to 256K", section "top-delta: Tearing
+        // Down "Global Synchronization" Too"): the topd best candidates and
+        // every candidate within delta of the best are both prefixes of the
+        // (score desc, page asc) order, so their union is the top
+        // max(topd, m), m = #{s >= s_max - delta} (threshold in fp32)
+        constexpr int W = NTHR / 32;
+        const int lane = tid & 31, warp = tid >> 5;
+        uint32_t km = __reduce_max_sync(0xffffffffu, kmax);
+        if (lane == 0) sc.red_max[warp] = km;
+        __syncthreads();
+        km = lane < W ? sc.red_max[lane] : 0u;
+        km = __reduce_max_sync(0xffffffffu, km);
+        __syncthreads();  // red_max is rewritten by the searches below
+        const float smax = (km & 0x80000000u) ? __uint_as_float(km & 0x7fffffffu)
+                                              : __uint_as_float(~km);
+        const uint32_t tk = order_key(smax - p.delta);
+        int c = 0;
+#pragma unroll
+        for (int k = 0; k < KPT; ++k) c += k < n_t && key[k] >= tk;
+        int m;
+        (void)block_excl_scan<NTHR>(c, sc, &m);
+        nsel = min(min(max(p.topd, m), p.budget), ncand);
+        if (nsel >= ncand) {
+            for (int i = tid; i < p.budget; i += NTHR) out[i] = i < ncand ? r.np + i : -1;
+            return;
+        }
+    }
+    for (int i = nsel + tid; i < p.budget; i += NTHR) out[i] = -1;
 
     // 1. tau from the threads' maxima
     uint32_t tau = 0u;

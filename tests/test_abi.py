@@ -26,7 +26,8 @@ def test_header_declares_the_boundary():
     names = declared()
     for want in ["slc_kv_append", "slc_build_page_meta", "slc_sparse_decode",
                  "slc_dense_decode", "slc_workspace_size", "slc_score_pages",
-                 "slc_select_pages", "slc_device_status", "slc_error_string"]:
+                 "slc_select_pages", "slc_select_pages_delta", "slc_sparse_decode_delta",
+                 "slc_device_status", "slc_error_string"]:
         assert want in names
 
 
@@ -112,6 +113,23 @@ def test_decode_argument_validation():
     assert lib.slc_select_pages(FAKE, 2, 10, FAKE, 1, 0, 0, 0, FAKE, None) == OK
     assert lib.slc_score_pages(FAKE, ctypes.byref(c), FAKE, 10, FAKE, 1, 8, -1, 0, FAKE,
                                None) == INVALID
+    # top-delta: d >= 0, cap >= 0, delta not NaN; nothing to do for cap 0 or batch 0
+    sd = lib.slc_select_pages_delta
+    assert sd(FAKE, 2, 10, FAKE, 1, 0, 0, -1, 1.0, 8, FAKE, None) == INVALID
+    assert sd(FAKE, 2, 10, FAKE, 1, 0, 0, 4, float("nan"), 8, FAKE, None) == INVALID
+    assert sd(FAKE, 2, 10, FAKE, 1, 0, 0, 4, 1.0, -1, FAKE, None) == INVALID
+    assert sd(FAKE, 2, 40000, FAKE, 1, 0, 0, 4, 1.0, 8, FAKE, None) == UNSUPPORTED
+    assert sd(FAKE, 2, 10, FAKE, 1, 0, 0, 4, float("inf"), 0, FAKE, None) == OK
+    assert sd(FAKE, 2, 10, FAKE, 0, 0, 0, 4, 1.0, 8, FAKE, None) == OK
+    dd = lib.slc_sparse_decode_delta
+    assert dd(FAKE, ctypes.byref(c), FAKE, 10, FAKE, 1, 8, 0, 0, -2, 1.0, 4, 0.0, FAKE, None,
+              FAKE, 1 << 40, None) == INVALID
+    assert dd(FAKE, ctypes.byref(c), FAKE, 10, FAKE, 1, 8, 0, 0, 2, float("nan"), 4, 0.0, FAKE,
+              None, FAKE, 1 << 40, None) == INVALID
+    assert dd(FAKE, ctypes.byref(c), FAKE, 10, FAKE, 1, 8, 0, 0, 2, 1.0, -4, 0.0, FAKE, None,
+              FAKE, 1 << 40, None) == INVALID
+    assert dd(FAKE, ctypes.byref(c), FAKE, 10, FAKE, 1, 8, 0, 0, 2, 1.0, 4, 0.0, FAKE, None,
+              FAKE, 100, None) == WORKSPACE
     assert lib.slc_device_status(None, None) == INVALID
     for stage in (0, 3, -1):  # only stages 1 and 2 exist
         assert lib.slc_sparse_decode_stage(stage, FAKE, ctypes.byref(c), FAKE, 10, FAKE, 1, 8, 0,

@@ -596,3 +596,76 @@ def test_fp8_meta_decode_parity(name):
     check_selection(x, sel, x.prefix, x.window, x.budget, scores=so)
     check_needles(x, sel)
     check_output(x, out, x.prefix, x.window, sel)
+
+
+# ------------------------------------------------------------------ top-delta
+
+def test_select_delta_exact_on_given_scores():
+    """Top-delta selection kernel against the oracle on scores of a 0.25 grid
+    (exact in fp32, so the fp32 threshold s_max - delta equals the oracle's):
+    bit-exact, over ties, caps below and above the union, d = 0, a negative
+    and an infinite delta, and unit sizes on both of the kernel's paths."""
+    import sparse_long_context_max_b200 as slc
+    rng = np.random.default_rng(12)
+    for ncand, d, delta, cap in [(50, 7, 1.0, 20), (50, 7, 1.0, 3), (4000, 128, 0.5, 300),
+                                 (16120, 256, 2.0, 512), (16120, 0, 0.75, 64),
+                                 (16120, 16, -1.0, 64), (900, 4, float("inf"), 1000),
+                                 (30000, 200, 1.5, 700), (9, 3, 0.25, 9)]:
+        B, hkv = 2, 3
+        L = 16 * (ncand + 2)
+        scores = np.full((B, hkv, ncand + 2), np.nan, dtype=np.float32)
+        scores[:, :, 1:ncand + 1] = np.round(rng.standard_normal((B, hkv, ncand)) * 8) / 4
+        sl = torch.tensor([L, L], dtype=torch.int32)
+        sel = slc.select_pages_delta(torch.from_numpy(scores).cuda(), sl.cuda(), 16, 16, d,
+                                     delta, cap)
+        want, _ = oracle.select_pages_delta(scores.astype(np.float64), sl, 16, 16, d, delta, cap)
+        np.testing.assert_array_equal(sel.cpu().numpy(), want, err_msg=str((ncand, d, delta, cap)))
+
+
+def check_selection_delta(x, sel_gpu, d, delta, cap, scores):
+    """GPU top-delta selection == the oracle's, except pages whose oracle
+    score is within TIE_BAND (relative to the best score) of one of the two
+    boundaries: the d-th best score and s_max - delta."""
+    sel_o, nsel_o = oracle.select_pages_delta(scores, x.seq_lens, x.prefix, x.window, d, delta,
+                                              cap)
+    B, hkv, _ = sel_o.shape
+    for b in range(B):
+        n, np_, ws = oracle.page_ranges(int(x.seq_lens[b]), x.prefix, x.window)
+        for h in range(hkv):
+            cand = scores[b, h, np_:ws]
+            smax = float(cand.max())
+            order = np.sort(cand)[::-1]
+            dth = float(order[min(d, len(order)) - 1]) if d > 0 else smax
+            o = set(int(p) for p in sel_o[b, h] if p >= 0)
+            g = [int(p) for p in sel_gpu[b, h]]
+            k = len([p for p in g if p >= 0])
+            assert g[k:] == [-1] * (cap - k) and g[:k] == sorted(g[:k]), (b, h)
+            for p in o ^ set(g[:k]):
+                s = scores[b, h, p]
+                near = min(abs(s - dth), abs(s - (smax - delta)))
+                assert near <= TIE_BAND * abs(smax), (b, h, p, s, smax)
+
+
+@pytest.mark.parametrize("name,d,delta,cap", [("tiny", 8, 2.0, 64), ("decode256k", 64, 40.0, 512),
+                                              ("ragged", 16, 25.0, 128)])
+def test_sparse_decode_delta_parity(name, d, delta, cap):
+    """The top-delta decode step (scores, top-delta selection, attention over
+    prefix + window + selection): the selection against the oracle's on the
+    oracle's scores within the tie bands, every needle page selected, and
+    the output against the oracle attending the GPU's selection."""
+    import sparse_long_context_max_b200 as slc
+    x = synth.make_inputs(W[name], fill="nan" if name == "ragged" else "zero")
+    dv = Dev(x)
+    B, hq, D = x.q.shape
+    hkv = x.k_cache.shape[1]
+    sel = torch.full((B, hkv, cap), -7, dtype=torch.int32, device="cuda")
+    out = slc.sparse_decode_delta(dv.q, dv.cache, dv.bt, dv.sl, x.prefix, x.window, d, delta,
+                                  cap, selected_out=sel)
+    torch.cuda.synchronize()
+    assert slc.device_status() == 0
+    sel = sel.cpu().numpy()
+    so = oracle_scores(x, x.prefix, x.window)
+    check_selection_delta(x, sel, d, delta, cap, so)
+    if name != "ragged":  # the needle pages top the scores: within the top d
+        check_needles(x, sel)
+    check_output(x, out.cpu(), x.prefix, x.window, sel)
