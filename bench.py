@@ -611,6 +611,28 @@ def run_ours(args, rank, world, local):
         assert slc.device_status() == 0
         del g8, W8
         torch.cuda.empty_cache()
+        # the same step with the top-delta selection (the top d pages plus every
+        # page within delta of the best, at most cap), through its four kernels
+        W9 = Workload("decode256k")
+        td, tdelta, tcap = 128, 40.0, 512
+        sel9 = torch.full((W9.q.shape[0], W9.wl.hkv, tcap), -1, dtype=torch.int32, device="cuda")
+        ws9 = torch.empty(slc.workspace_size(W9.q.shape[0], W9.q.shape[1], W9.wl.hkv,
+                                             W9.wl.head_dim, W9.bt.shape[1], tcap),
+                          dtype=torch.uint8, device="cuda")
+        g9 = graph_of(lambda: slc.sparse_decode_delta(W9.q, W9.cache, W9.bt, W9.sl, y.prefix,
+                                                      y.window, td, tdelta, tcap, out=W9.out,
+                                                      selected_out=sel9, workspace=ws9))
+        sp9 = timed(g9.replay, max(reps, 32), None)
+        nsel9 = (sel9 >= 0).sum(dim=2).float().mean().item()
+        b9 = algorithmic_bytes(lens256, y.wl.hq, y.wl.hkv, y.wl.head_dim, y.prefix, y.window,
+                               int(round(nsel9)))
+        top256.update({"decode256k_topdelta_us": round(sp9 * 1e3, 2),
+                       "decode256k_topdelta_config": {"d": td, "delta": tdelta, "cap": tcap},
+                       "decode256k_topdelta_mean_selected_pages": round(nsel9, 1),
+                       "decode256k_topdelta_hbm_gbs": round(b9[0] / (sp9 * 1e-3) / 1e9, 1)})
+        assert slc.device_status() == 0
+        del g9, W9, ws9, sel9
+        torch.cuda.empty_cache()
         if not args.no_also:
             for name in ("tiny", "ragged"):
                 Wx = Workload(name)
