@@ -13,8 +13,10 @@ nearest Full layer before it, together with its own prefix and window.
 q, k and v per layer, the positions, the lengths, the outputs and the Full
 layers' selections) and runs, per layer, ``kv_append`` then that layer's
 decode through the C ABI; ``capture()`` records the whole step as one CUDA
-graph.  This module orders calls only: every step of the path runs in the
-library's kernels.
+graph.  The per-step inputs live in one device byte buffer, so a caller
+feeding them from the host moves them with a single copy (``host_buffers``,
+``run_from_host``).  This module orders calls only: every step of the path
+runs in the library's kernels.
 """
 from __future__ import annotations
 
@@ -26,7 +28,59 @@ import torch
 from . import (PagedCache, dense_decode, kv_append, sparse_attend, sparse_decode,
                workspace_size)
 
-__all__ = ["LayerSpec", "index_reuse", "DecodeStep"]
+__all__ = ["LayerSpec", "index_reuse", "DecodeStep", "StepIO", "packed_layout"]
+
+_ALIGN = 256  # byte alignment of every tensor inside the packed input buffer
+
+
+def packed_layout(num_layers: int, batch: int, num_q_heads: int, num_kv_heads: int,
+                  head_dim: int):
+    """Byte layout of a step's inputs in one buffer: (name, offset, shape,
+    dtype) for q (bf16 [layers][B][Hq][D]), k_new and v_new (bf16
+    [layers][B][Hkv][D]), positions and seq_lens (int32 [B]), each at an
+    offset that is a multiple of 256 bytes; and the total size."""
+    items = [("q", (num_layers, batch, num_q_heads, head_dim), torch.bfloat16),
+             ("k_new", (num_layers, batch, num_kv_heads, head_dim), torch.bfloat16),
+             ("v_new", (num_layers, batch, num_kv_heads, head_dim), torch.bfloat16),
+             ("positions", (batch,), torch.int32),
+             ("seq_lens", (batch,), torch.int32)]
+    out, off = [], 0
+    for name, shape, dt in items:
+        n = 1
+        for v in shape:
+            n *= v
+        out.append((name, off, shape, dt))
+        off += -(-n * torch.empty((), dtype=dt).element_size() // _ALIGN) * _ALIGN
+    return out, off
+
+
+def _views(buf: torch.Tensor, layout) -> dict:
+    views = {}
+    for name, off, shape, dt in layout:
+        n = 1
+        for v in shape:
+            n *= v
+        nb = n * torch.empty((), dtype=dt).element_size()
+        views[name] = buf[off:off + nb].view(dt).view(shape)
+    return views
+
+
+@dataclasses.dataclass
+class StepIO:
+    """Pinned host buffers mirroring a DecodeStep's inputs and outputs.
+
+    inputs     uint8, the packed bytes (copied to the device in one copy)
+    q, k_new, v_new, positions, seq_lens   views into ``inputs``
+    out        fp32 [layers][B][Hq][D], filled by ``run_from_host``
+    """
+
+    inputs: torch.Tensor
+    q: torch.Tensor
+    k_new: torch.Tensor
+    v_new: torch.Tensor
+    positions: torch.Tensor
+    seq_lens: torch.Tensor
+    out: torch.Tensor
 
 
 @dataclasses.dataclass(frozen=True)
@@ -102,11 +156,11 @@ class DecodeStep:
                 last_full = i
                 self.full_of.append(i)
         L = len(self.specs)
-        self.q = torch.zeros((L, B, num_q_heads, D), dtype=torch.bfloat16, device=dev)
-        self.k_new = torch.zeros((L, B, hkv, D), dtype=torch.bfloat16, device=dev)
-        self.v_new = torch.zeros((L, B, hkv, D), dtype=torch.bfloat16, device=dev)
-        self.positions = torch.zeros((B,), dtype=torch.int32, device=dev)
-        self.seq_lens = torch.zeros((B,), dtype=torch.int32, device=dev)
+        self.layout, nbytes = packed_layout(L, B, num_q_heads, hkv, D)
+        self.inputs = torch.zeros((nbytes,), dtype=torch.uint8, device=dev)
+        v = _views(self.inputs, self.layout)
+        self.q, self.k_new, self.v_new = v["q"], v["k_new"], v["v_new"]
+        self.positions, self.seq_lens = v["positions"], v["seq_lens"]
         self.out = torch.zeros((L, B, num_q_heads, D), dtype=torch.float32, device=dev)
         self.selected = {i: torch.full((B, hkv, max(s.budget, 1)), -1, dtype=torch.int32,
                                        device=dev)[:, :, : s.budget].contiguous()
@@ -158,3 +212,19 @@ class DecodeStep:
         if self.graph is None:
             self.capture()
         self.graph.replay()
+
+    def host_buffers(self) -> StepIO:
+        """Pinned host buffers laid out like this step's inputs and output."""
+        buf = torch.zeros(self.inputs.shape, dtype=torch.uint8).pin_memory()
+        v = _views(buf, self.layout)
+        out = torch.zeros(self.out.shape, dtype=torch.float32).pin_memory()
+        return StepIO(buf, v["q"], v["k_new"], v["v_new"], v["positions"], v["seq_lens"], out)
+
+    def run_from_host(self, io: StepIO):
+        """Issue, on the current stream: one host-to-device copy of
+        ``io.inputs``, the step (its graph), one device-to-host copy of the
+        outputs into ``io.out``.  Asynchronous: synchronise before reading
+        ``io.out`` or rewriting ``io.inputs``."""
+        self.inputs.copy_(io.inputs, non_blocking=True)
+        self.replay()
+        io.out.copy_(self.out, non_blocking=True)

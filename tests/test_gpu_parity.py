@@ -461,8 +461,9 @@ def test_layers131k_sampled_layers():
 
 def test_layers131k_graph_step_all_layers():
     """One decode step of the 15-layer plan at 131072 tokens (d 256), replayed
-    from its CUDA graph: per layer the new token's append, then the layer's
-    decode.  Cross-layer reuse is on ("IndexCache: cross-layer reuse speeds
+    from its CUDA graph with the inputs copied in from pinned host buffers
+    and the outputs copied back: per layer the new token's append, then the
+    layer's decode.  Cross-layer reuse is on ("IndexCache: cross-layer reuse speeds
     30B prefill 1.82x": Full layers select, Shared layers attend the nearest
     Full layer's selection with their own window).  Checked per layer: the
     appended token landed, Full layers' selections against the oracle's
@@ -486,16 +487,18 @@ def test_layers131k_graph_step_all_layers():
     del k0, v0
     step = P.DecodeStep(caches, bt, specs, wl.prefix, wl.hq)
     toks = [synth.step_tokens(wl, 1, layer=i) for i in range(len(specs))]
+    io = step.host_buffers()  # the inputs travel as one packed host-to-device copy
     for i, (q, kn, vn) in enumerate(toks):
-        step.q[i].copy_(q)
-        step.k_new[i].copy_(kn)
-        step.v_new[i].copy_(vn)
-    step.positions.copy_(x.seq_lens)
-    step.seq_lens.copy_(x.seq_lens + 1)
-    step.capture()
-    step.replay()  # the append writes the same slot again: idempotent
+        io.q[i].copy_(q)
+        io.k_new[i].copy_(kn)
+        io.v_new[i].copy_(vn)
+    io.positions.copy_(x.seq_lens)
+    io.seq_lens.copy_(x.seq_lens + 1)
+    step.run_from_host(io)  # captures on first use, then replays
+    step.run_from_host(io)  # the append writes the same slot again: idempotent
     torch.cuda.synchronize()
     assert slc.device_status() == 0
+    assert torch.equal(io.out, step.out.cpu())
     lens1 = x.seq_lens + 1
     for i, s in enumerate(specs):
         q, kn, vn = toks[i]
