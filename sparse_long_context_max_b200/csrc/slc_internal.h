@@ -43,8 +43,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 constexpr int kMaxAttendChunks = 1024;
 
 // Cluster sizes the finishing kernel may be launched with.
-constexpr int kFinishClusters[] = {16, 8, 7, 6, 5, 4};
-constexpr int kNumFinishClusters = 6;
+constexpr int kFinishClusters[] = {16, 12, 10, 9, 8, 7, 6, 5, 4};
+constexpr int kNumFinishClusters = 9;
 
 // Per-device launch settings, looked up once per device (with that device
 // current) by slc_api.cu and passed to every launch.
