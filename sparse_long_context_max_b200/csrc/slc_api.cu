@@ -51,6 +51,12 @@ int device_cfg(const DeviceCfg** out) {
         if (e != cudaSuccess) return note_cuda(e);
         e = cudaGetSymbolAddress(reinterpret_cast<void**>(&c.status), slc_status_word);
         if (e != cudaSuccess) return note_cuda(e);
+        int win = 0;  // no access-policy windows where the attribute is not there
+        if (cudaDeviceGetAttribute(&win, cudaDevAttrMaxAccessPolicyWindowSize, dev) != cudaSuccess) {
+            (void)cudaGetLastError();
+            win = 0;
+        }
+        c.max_window = win > 0 ? (size_t)win : 0;
         if ((e = setup_score(c)) != cudaSuccess) return note_cuda(e, "setup score");
         if ((e = setup_select(c)) != cudaSuccess) return note_cuda(e, "setup select");
         if ((e = setup_attend(c)) != cudaSuccess) return note_cuda(e, "setup attend");

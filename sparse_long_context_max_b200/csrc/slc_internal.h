@@ -10,32 +10,58 @@
 
 namespace slc {
 
+// An address range a launch reads once, front to back: its L2 lines are
+// marked evict-first (an access-policy window with the streaming property),
+// so that the stream does not push out what the next kernels reuse (their
+// code, the workspace).  bytes = 0: none.
+struct StreamingRange {
+    const void* base = nullptr;
+    size_t bytes = 0;
+};
+
 // Launch with programmatic stream serialization: the kernel may start while
 // the preceding kernel in the stream is still running; it calls
 // grid_dep_wait() before touching anything that kernel produces.
 // cluster > 1 also sets the thread-block cluster size (x).
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t stream, int cluster, Args&&... args) {
+cudaError_t launch_pdl_streaming(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t stream, int cluster, StreamingRange range,
+                                 Args&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[3];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     int n = 1;
     if (cluster > 1) {
-        attr[1].id = cudaLaunchAttributeClusterDimension;
-        attr[1].val.clusterDim.x = cluster;
-        attr[1].val.clusterDim.y = 1;
-        attr[1].val.clusterDim.z = 1;
-        n = 2;
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    if (range.bytes > 0) {
+        attr[n].id = cudaLaunchAttributeAccessPolicyWindow;
+        attr[n].val.accessPolicyWindow.base_ptr = const_cast<void*>(range.base);
+        attr[n].val.accessPolicyWindow.num_bytes = range.bytes;
+        attr[n].val.accessPolicyWindow.hitRatio = 1.0f;
+        attr[n].val.accessPolicyWindow.hitProp = cudaAccessPropertyStreaming;
+        attr[n].val.accessPolicyWindow.missProp = cudaAccessPropertyStreaming;
+        ++n;
     }
     cfg.attrs = attr;
     cfg.numAttrs = n;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, int cluster, Args&&... args) {
+    return launch_pdl_streaming(kernel, grid, block, smem, stream, cluster, StreamingRange{},
+                                std::forward<Args>(args)...);
 }
 
 // Upper bound on the number of attention CTAs (chunks) of one launch; sizes
@@ -56,7 +82,21 @@ struct DeviceCfg {
     int occ_stream[2];      // stream_kernel CTAs per SM (D = 128, 256)
     int occ_attend[3];      // attend_kernel CTAs per SM (D = 128 sparse shape, D = 128 dense, D = 256)
     int finish_clusters[2][kNumFinishClusters];  // co-resident finish clusters (D, cluster size)
+    size_t max_window;      // largest L2 access-policy window, bytes (0: none)
 };
+
+// The page metadata as a streaming range for the launches that scan it: the
+// whole array, or its first max_window bytes.
+inline StreamingRange metadata_range(const void* meta, long long num_pages, int hkv, int head_dim,
+                                     int meta_format, const DeviceCfg& d) {
+    StreamingRange r;
+    if (meta == nullptr || d.max_window == 0) return r;
+    const size_t elem = meta_format == SLC_META_FP8_E4M3 ? 1 : 2;
+    const size_t bytes = (size_t)num_pages * hkv * 2 * head_dim * elem;
+    r.base = meta;
+    r.bytes = bytes < d.max_window ? bytes : d.max_window;
+    return r;
+}
 
 cudaError_t setup_score(DeviceCfg& d);
 cudaError_t setup_select(DeviceCfg& d);

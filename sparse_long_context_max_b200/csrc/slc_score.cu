@@ -84,9 +84,12 @@ cudaError_t setup_one(int* occ) {
 }
 
 template <int D, bool FP8>
-cudaError_t run(const ScoreParams& p, int occ, int num_sms, cudaStream_t stream) {
-    return launch_pdl(score_kernel<D, FP8>, dim3(num_sms * occ), dim3(kScoreWarps * 32),
-                      ScoreCfg<D, FP8>::SMEM, stream, 1, p);
+cudaError_t run(const ScoreParams& p, int occ, const DeviceCfg& d, cudaStream_t stream) {
+    // the metadata is read once per call: streamed through L2
+    return launch_pdl_streaming(score_kernel<D, FP8>, dim3(d.num_sms * occ),
+                                dim3(kScoreWarps * 32), ScoreCfg<D, FP8>::SMEM, stream, 1,
+                                metadata_range(p.meta, p.num_pages, p.hkv, D, p.meta_format, d),
+                                p);
 }
 
 }  // namespace
@@ -104,10 +107,10 @@ cudaError_t launch_score(const ScoreParams& p, int head_dim, const DeviceCfg& d,
                          cudaStream_t stream) {
     const bool fp8 = p.meta_format == SLC_META_FP8_E4M3;
     if (head_dim == 128)
-        return fp8 ? run<128, true>(p, d.occ_score[0], d.num_sms, stream)
-                   : run<128, false>(p, d.occ_score[0], d.num_sms, stream);
-    return fp8 ? run<256, true>(p, d.occ_score[1], d.num_sms, stream)
-               : run<256, false>(p, d.occ_score[1], d.num_sms, stream);
+        return fp8 ? run<128, true>(p, d.occ_score[0], d, stream)
+                   : run<128, false>(p, d.occ_score[0], d, stream);
+    return fp8 ? run<256, true>(p, d.occ_score[1], d, stream)
+               : run<256, false>(p, d.occ_score[1], d, stream);
 }
 
 }  // namespace slc

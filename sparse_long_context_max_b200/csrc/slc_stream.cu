@@ -122,9 +122,14 @@ cudaError_t setup_one(int* occ) {
 }
 
 template <int D, bool FP8>
-cudaError_t run(StreamParams& p, int blocks, cudaStream_t stream) {
-    return launch_pdl(stream_kernel<D, FP8>, dim3(blocks), dim3(StreamCfg<D>::NW * 32),
-                      StreamCfg<D>::SMEM, stream, 1, p);
+cudaError_t run(StreamParams& p, int blocks, const DeviceCfg& d, cudaStream_t stream) {
+    // the metadata is read once per call: streamed through L2
+    const StreamingRange meta =
+        p.sc.scores != nullptr ? metadata_range(p.sc.meta, p.sc.num_pages, p.sc.hkv, D,
+                                                p.sc.meta_format, d)
+                               : StreamingRange{};
+    return launch_pdl_streaming(stream_kernel<D, FP8>, dim3(blocks), dim3(StreamCfg<D>::NW * 32),
+                                StreamCfg<D>::SMEM, stream, 1, meta, p);
 }
 
 }  // namespace
@@ -154,8 +159,9 @@ cudaError_t launch_stream(StreamParams& p, int head_dim, const DeviceCfg& d,
     p.at.num_chunks = blocks;
     p.at.list = kListForced;
     const bool fp8 = p.sc.meta_format == SLC_META_FP8_E4M3;
-    if (d128) return fp8 ? run<128, true>(p, blocks, stream) : run<128, false>(p, blocks, stream);
-    return fp8 ? run<256, true>(p, blocks, stream) : run<256, false>(p, blocks, stream);
+    if (d128)
+        return fp8 ? run<128, true>(p, blocks, d, stream) : run<128, false>(p, blocks, d, stream);
+    return fp8 ? run<256, true>(p, blocks, d, stream) : run<256, false>(p, blocks, d, stream);
 }
 
 }  // namespace slc
