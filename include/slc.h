@@ -232,12 +232,13 @@ SLC_API int slc_sparse_attend(const void *q, const slc_cache_t *cache, const int
                       size_t workspace_bytes, slc_stream_t stream);
 
 /* One decode step with the top-delta selection in place of the fixed
- * budget: the candidate scores (slc_score_pages), the top-delta selection
- * (slc_select_pages_delta, into selected_out when given, else the
- * workspace), then attention over the prefix, window and selected pages and
- * the merge (as slc_sparse_attend): four kernels.  workspace >=
- * slc_workspace_size(..., budget = cap).  Other arguments as
- * slc_sparse_decode and slc_select_pages_delta. */
+ * budget: the two kernels of slc_sparse_decode, the finishing kernel setting
+ * each unit's selection size from its scores (the top d plus every candidate
+ * within delta of the best, at most cap; the same selection as
+ * slc_select_pages_delta on the same scores), written to selected_out when
+ * given (int32 [batch][num_kv_heads][cap], ascending, -1 padded).
+ * workspace >= slc_workspace_size(..., budget = cap).  Other arguments and
+ * errors as slc_sparse_decode and slc_select_pages_delta. */
 SLC_API int slc_sparse_decode_delta(const void *q, const slc_cache_t *cache,
                             const int32_t *block_table, int32_t max_pages_per_seq,
                             const int32_t *seq_lens, int32_t batch, int32_t num_q_heads,

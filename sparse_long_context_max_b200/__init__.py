@@ -37,7 +37,7 @@ PAGE = 16
 KERNELS_PER_CALL = {"sparse_decode": 2, "sparse_decode_stage": 1, "dense_decode": 2,
                     "sparse_attend": 2, "kv_append": 1,
                     "build_page_meta": 1, "score_pages": 1, "select_pages": 1,
-                    "select_pages_delta": 1, "sparse_decode_delta": 4}
+                    "select_pages_delta": 1, "sparse_decode_delta": 2}
 
 STATUS_BITS = {1: "bad page", 2: "bad length", 4: "bad selection", 8: "wait timeout"}
 

@@ -279,7 +279,7 @@ static int decode(int mode, const void* q, const slc_cache_t* cache,
                   const int32_t* seq_lens, int32_t batch, int32_t num_q_heads, int32_t prefix,
                   int32_t window, int32_t budget, float scale, float* out,
                   int32_t* selected_out, void* workspace, size_t workspace_bytes,
-                  cudaStream_t stream, int stage = 0) {
+                  cudaStream_t stream, int stage = 0, int topd = -1, float delta = 0.f) {
     const bool sparse = mode != 0;
     bool empty;
     int rc = check_decode(mode, q, cache, block_table, max_pages_per_seq, seq_lens, batch,
@@ -349,6 +349,8 @@ static int decode(int mode, const void* q, const slc_cache_t* cache,
     fp.budget = budget;
     fp.cand_stride = cs;
     fp.stream_scored = scoring ? 1 : 0;
+    fp.topd = mode == 1 ? topd : -1;
+    fp.delta = delta;
     e = launch_finish(fp, D, *dev, stream);
     return e == cudaSuccess ? SLC_OK : note_cuda(e, "finish");
 }
@@ -397,24 +399,11 @@ int slc_sparse_decode_delta(const void* q, const slc_cache_t* cache, const int32
     if (rc) return rc;
     if (d < 0 || delta != delta) return SLC_ERR_INVALID_ARG;
     if (empty) return SLC_OK;
-    if (!workspace || !aligned16(workspace)) return SLC_ERR_INVALID_ARG;
-    const int hkv = cache->num_kv_heads;
-    const WorkspaceLayout w =
-        workspace_layout(batch, num_q_heads, hkv, cache->head_dim, max_pages_per_seq, cap);
-    if (workspace_bytes < w.total) return SLC_ERR_WORKSPACE;
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    // scores by page in the scores region (rows of max_pages floats fit its
-    // rows of cand_stride), the selection in selected_out or the workspace
-    float* scores = reinterpret_cast<float*>(ws + w.scores);
-    int32_t* sel = selected_out ? selected_out : reinterpret_cast<int32_t*>(ws + w.selected);
-    rc = slc_score_pages(q, cache, block_table, max_pages_per_seq, seq_lens, batch, num_q_heads,
-                         prefix, window, scores, stream);
-    if (rc) return rc;
-    rc = slc_select_pages_delta(scores, hkv, max_pages_per_seq, seq_lens, batch, prefix, window,
-                                d, delta, cap, sel, stream);
-    if (rc) return rc;
-    return decode(2, q, cache, block_table, max_pages_per_seq, seq_lens, batch, num_q_heads,
-                  prefix, window, cap, scale, out, sel, workspace, workspace_bytes, stream);
+    // the two kernels of slc_sparse_decode; the finishing kernel sets each
+    // unit's selection size from its scores
+    return decode(1, q, cache, block_table, max_pages_per_seq, seq_lens, batch, num_q_heads,
+                  prefix, window, cap, scale, out, selected_out, workspace, workspace_bytes,
+                  stream, 0, d, delta);
 }
 
 int slc_dense_decode(const void* q, const slc_cache_t* cache, const int32_t* block_table,

@@ -50,6 +50,17 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Top-delta threshold ("Faster Than Flash: Fudan FFD Hits 11.6x Kernel
+// Speedup, Pushes Long-Context Decoding to 256K", section "top-delta: Tearing
+// Down "Global Synchronization" Too"): the order key of s_max - delta, s_max
+// the score whose key is kmax, computed in fp32.  A candidate is within delta
+// of the best iff its key is >= this one.
+__device__ __forceinline__ uint32_t delta_threshold_key(uint32_t kmax, float delta) {
+    const float smax = (kmax & 0x80000000u) ? __uint_as_float(kmax & 0x7fffffffu)
+                                            : __uint_as_float(~kmax);
+    return order_key(smax - delta);
+}
+
 // ---------------------------------------------------------------- E4M3
 // 8-bit floats E4M3 (OCP "FN": sign, 4 exponent bits with bias 7, 3
 // mantissa bits; exponent field 0 is subnormal, m/8 * 2^-6; no infinities;

@@ -78,6 +78,7 @@ struct alignas(16) FinishShared {
     int scount;          // this CTA's survivors (read remotely)
     int soff[kMaxCluster + 1];  // survivors of the ranks before each rank
     int bcnt[2][16];     // bisection counts per trial digit, double-buffered
+    int dcount;          // this CTA's keys within delta of the best (read remotely)
     long long k0, k1;    // the unit's streaming-partial chunks
     uint64_t bar;        // the score copy
 };
@@ -500,10 +501,15 @@ __global__ void __launch_bounds__(FinishCfg<D>::NT, FinishCfg<D>::MIN_BLOCKS)
         const int L = checked_len(a.seq_lens, b, a.max_pages, a.status);
         const PageRanges r = page_ranges(L, a.prefix, a.window);
         const int ncand = r.ws - r.np;
-        const int nsel = min(p.budget, ncand);
+        int nsel = min(p.budget, ncand);
         int32_t* sel_row = p.selected ? p.selected + (long long)u * p.budget : nullptr;
         int32_t* phys_row = p.sel_phys + (long long)u * p.budget;
-        const bool selecting = p.scores != nullptr && nsel > 0 && nsel < ncand;
+        // top-delta: the unit's selection size comes from its scores, unless
+        // topd alone settles it (topd >= ncand, or budget <= topd: the top
+        // min(budget, ncand)); the tile maxima always come with the scores
+        const bool by_delta = p.scores != nullptr && p.topd >= 0 && p.topd < ncand &&
+                              p.topd < p.budget;
+        bool selecting = p.scores != nullptr && nsel > 0 && (by_delta || nsel < ncand);
         // this CTA's slice of the candidates
         const int pc = ((ncand + C - 1) / C + 3) / 4 * 4;
         const int c0 = min(rank * pc, ncand);
@@ -568,15 +574,16 @@ __global__ void __launch_bounds__(FinishCfg<D>::NT, FinishCfg<D>::MIN_BLOCKS)
         // cluster-wide radix search over all keys.
         bool local_list = false;  // the selected list is in this CTA's shared memory
         int2* list = reinterpret_cast<int2*>(keys);  // (page, physical page)
+        const int ntiles = (ncand + kSelTile - 1) / kSelTile;
+        uint32_t* tkeys = reinterpret_cast<uint32_t*>(smem);  // the ring area
         if (selecting) {
-            const int ntiles = (ncand + kSelTile - 1) / kSelTile;
-            const bool bound = p.tile_max != nullptr && ntiles >= nsel &&
-                               nsel <= kMaxCandidates / C;  // the list fits keys + phys
-            uint32_t* tkeys = reinterpret_cast<uint32_t*>(smem);  // the ring area
-            if (cnt > 0 || bound) {
+            // the tile maxima serve the survivor path's bound and top-delta's s_max
+            const bool tiles_in = p.tile_max != nullptr &&
+                                  (by_delta || (ntiles >= nsel && nsel <= kMaxCandidates / C));
+            if (cnt > 0 || tiles_in) {
                 if (tid == 0) {
                     const uint32_t kb = cnt > 0 ? (uint32_t)((cnt + 3) / 4 * 4) * 4 : 0u;
-                    const uint32_t tb = bound ? (uint32_t)((ntiles + 3) / 4 * 4) * 4 : 0u;
+                    const uint32_t tb = tiles_in ? (uint32_t)((ntiles + 3) / 4 * 4) * 4 : 0u;
                     fence_proxy_async_smem();  // earlier generic accesses of keys[] first
                     mbar_arrive_expect_tx(&sh.bar, kb + tb);
                     if (kb)
@@ -596,6 +603,49 @@ __global__ void __launch_bounds__(FinishCfg<D>::NT, FinishCfg<D>::MIN_BLOCKS)
                     keys[i] = order_key(__uint_as_float(keys[i]));
             }
             __syncthreads();
+            if (by_delta) {
+                // top-delta ("Faster Than Flash: Fudan FFD Hits 11.6x Kernel
+                // Speedup, Pushes Long-Context Decoding to 256K", section
+                // "top-delta: Tearing Down "Global Synchronization" Too"): the
+                // top topd and the candidates within delta of the best are both
+                // prefixes of the (score desc, page asc) order, so their union
+                // is the top max(topd, m), m = #{s >= s_max - delta}.  s_max is
+                // the largest tile maximum (every CTA holds them all); m sums
+                // the CTAs' counts
+                uint32_t km = 0u;
+                for (int t = tid; t < ntiles; t += NT) km = max(km, tkeys[t]);
+                km = __reduce_max_sync(0xffffffffu, km);
+                if (lane == 0) sh.red_max[warp] = km;
+                __syncthreads();
+#pragma unroll
+                for (int w2 = 0; w2 < NW; ++w2) km = max(km, sh.red_max[w2]);
+                const uint32_t tk = delta_threshold_key(km, p.delta);
+                int c = 0;
+                for (int i = tid; i < cnt; i += NT) c += keys[i] >= tk ? 1 : 0;
+                c = __reduce_add_sync(0xffffffffu, c);
+                if (lane == 0) sh.wcnt[warp] = make_int2(c, 0);
+                __syncthreads();
+                if (tid == 0) {
+                    int s2 = 0;
+#pragma unroll
+                    for (int w2 = 0; w2 < NW; ++w2) s2 += sh.wcnt[w2].x;
+                    sh.dcount = s2;
+                }
+                cl.sync();  // every CTA's count is published
+                const int rr = lane & (kMaxCluster - 1);
+                const int cr = remote(cl, &sh.dcount, rr, C);
+                const int m =
+                    __reduce_add_sync(0xffffffffu, lane < kMaxCluster && rr < C ? cr : 0);
+                nsel = min(min(max(p.topd, m), p.budget), ncand);
+                if (nsel == 0 || nsel >= ncand) {  // none, or every candidate: no search
+                    selecting = false;
+                    cp_async_wait<0>();  // this thread's phys[] copies, unused now
+                }
+            }
+        }
+        if (selecting) {
+            const bool bound = p.tile_max != nullptr && ntiles >= nsel &&
+                               nsel <= kMaxCandidates / C;  // the list fits keys + phys
             bool fast = false;
             if (bound) {
                 // tau: each warp's ceil(nsel / NW)-th largest tile maximum

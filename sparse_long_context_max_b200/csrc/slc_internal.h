@@ -202,6 +202,10 @@ struct FinishParams {
     int32_t* selected;      // [units][budget] out: ascending, -1 padded (scores != null)
     int32_t* sel_phys;      // [units][budget] workspace: physical page of each selected entry
     int budget, cand_stride;
+    // top-delta selection (topd >= 0): per unit the top max(topd, m) candidates,
+    // m = #{s >= s_max - delta}, at most budget; topd < 0: the top budget
+    int topd;
+    float delta;
 };
 
 // Workspace carve-up shared by the API and the size query.

@@ -331,9 +331,7 @@ __device__ void select_unit(const SelectParams& p, int u, Scratch<NTHR>& sc, uin
         km = lane < W ? sc.red_max[lane] : 0u;
         km = __reduce_max_sync(0xffffffffu, km);
         __syncthreads();  // red_max is rewritten by the searches below
-        const float smax = (km & 0x80000000u) ? __uint_as_float(km & 0x7fffffffu)
-                                              : __uint_as_float(~km);
-        const uint32_t tk = order_key(smax - p.delta);
+        const uint32_t tk = delta_threshold_key(km, p.delta);
         int c = 0;
 #pragma unroll
         for (int k = 0; k < KPT; ++k) c += k < n_t && key[k] >= tk;

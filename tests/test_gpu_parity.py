@@ -649,6 +649,35 @@ def check_selection_delta(x, sel_gpu, d, delta, cap, scores):
                 assert near <= TIE_BAND * abs(smax), (b, h, p, s, smax)
 
 
+@pytest.mark.parametrize("d,delta,cap", [(8, 3.0, 64), (8, 3.0, 6), (0, -1.0, 32), (5, 0.0, 40),
+                                         (0, float("inf"), 300), (400, 1.0, 500), (3, 1e30, 20),
+                                         (16, 6.0, 0)])
+def test_sparse_decode_delta_matches_the_standalone_selection(d, delta, cap):
+    """The top-delta decode step sets each unit's selection size inside the
+    finishing kernel; on the same scores (the scoring code is shared) its
+    selection equals the standalone top-delta kernel's bit for bit, over the
+    edges: d past the candidates, cap below d, nothing within a negative
+    delta of the best with d = 0, every candidate (delta = inf), cap 0.  The
+    output is checked against the oracle attending that selection."""
+    import sparse_long_context_max_b200 as slc
+    x = small(3, 8, 2, 128, [4096, 2000, 300], prefix=32, window=256, seed=41, needles=4)
+    dv = Dev(x)
+    B, hq, D = x.q.shape
+    hkv = x.k_cache.shape[1]
+    width = max(cap, 1)
+    sel = torch.full((B, hkv, width), -7, dtype=torch.int32, device="cuda")[:, :, :cap]
+    sel = sel.contiguous()
+    out = slc.sparse_decode_delta(dv.q, dv.cache, dv.bt, dv.sl, x.prefix, x.window, d, delta,
+                                  cap, selected_out=sel if cap > 0 else None)
+    scores = slc.score_pages(dv.q, dv.cache, dv.bt, dv.sl, x.prefix, x.window)
+    want = slc.select_pages_delta(scores, dv.sl, x.prefix, x.window, d, delta, cap) \
+        if cap > 0 else torch.empty((B, hkv, 0), dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    assert slc.device_status() == 0
+    np.testing.assert_array_equal(sel.cpu().numpy(), want.cpu().numpy())
+    check_output(x, out.cpu().double().numpy(), x.prefix, x.window, sel.cpu().numpy())
+
+
 @pytest.mark.parametrize("name,d,delta,cap", [("tiny", 8, 2.0, 64), ("decode256k", 64, 40.0, 512),
                                               ("ragged", 16, 25.0, 128)])
 def test_sparse_decode_delta_parity(name, d, delta, cap):
