@@ -62,7 +62,6 @@ struct FinishCfg {
 };
 
 constexpr int kBins = 256;       // 8-bit digits
-constexpr int kBisectKeys = 16;  // keys per lane of the register bisection (up to 512 keys)
 constexpr int kMaxCluster = 16;  // the largest cluster size launched
 
 // Shared memory: rings | bars | nvalid | keys[cap] | phys[cap] | FinishShared
@@ -77,7 +76,6 @@ struct alignas(16) FinishShared {
     int2 counts;         // this CTA's (keys > T, keys == T) (read remotely)
     int scount;          // this CTA's survivors (read remotely)
     int soff[kMaxCluster + 1];  // survivors of the ranks before each rank
-    int bcnt[2][16];     // bisection counts per trial digit, double-buffered
     int dcount;          // this CTA's keys within delta of the best (read remotely)
     long long k0, k1;    // the unit's streaming-partial chunks
     uint64_t bar;        // the score copy
@@ -387,78 +385,6 @@ __device__ __noinline__ void cta_kth(const uint32_t* keys, int stride, int n, in
     }
 }
 
-// The k-th largest of n <= 32 * NK keys held by this CTA (keys[i * stride],
-// i < n), by a multi-threshold bisection: every warp holds all the keys in
-// registers; from the highest bit where the smallest and largest keys
-// differ, each step fixes up to four bits at once (warp w counts the keys >=
-// T | d << s for its two trial digits d = 2w + 1, 2w + 2; one barrier
-// publishes the fifteen counts; every thread takes the largest digit whose
-// count is >= k).  T ends as the k-th largest key; ties = k - #(keys > T).
-// Same result form as cta_kth: the k largest keys are the keys > T plus the
-// first `ties` keys == T in index order.  1 <= k <= n.
-template <int NT, int NK>
-__device__ __noinline__ void cta_kth_bisect(const uint32_t* keys, int stride, int n, int k,
-                                            FinishShared& sh, uint32_t* T_out,
-                                            int* ties_out) {
-    static_assert(NT == 256, "eight warps: two trial digits each cover a 4-bit digit");
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint32_t v[NK];
-    uint32_t kmin = 0xffffffffu, kmax = 0u;
-#pragma unroll
-    for (int c = 0; c < NK; ++c) {
-        const int i = 32 * c + lane;
-        v[c] = i < n ? keys[i * stride] : 0u;
-        if (i < n) {
-            kmin = min(kmin, v[c]);
-            kmax = max(kmax, v[c]);
-        }
-    }
-    kmin = __reduce_min_sync(0xffffffffu, kmin);
-    kmax = __reduce_max_sync(0xffffffffu, kmax);
-    if (kmin == kmax) {  // every key equal: the first k of them
-        *T_out = kmin;
-        *ties_out = k;
-        return;
-    }
-    const int hb = 31 - __clz(kmin ^ kmax);
-    uint32_t T = hb == 31 ? 0u : kmin & ~((2u << hb) - 1u);  // the bits every key shares
-    int buf = 0;
-    for (int bit = hb; bit >= 0;) {
-        const int w = min(bit + 1, 4);  // this step's digit width and shift
-        const int sft = bit + 1 - w;
-        const uint32_t nd = 1u << w;
-        const uint32_t d1 = 2u * warp + 1u, d2 = d1 + 1u;
-        const uint32_t t1 = T | (d1 << sft), t2 = T | (d2 << sft);
-        int c1 = 0, c2 = 0;
-#pragma unroll
-        for (int c = 0; c < NK; ++c) {
-            const bool live = 32 * c + lane < n;
-            c1 += live && v[c] >= t1 ? 1 : 0;
-            c2 += live && v[c] >= t2 ? 1 : 0;
-        }
-        c1 = __reduce_add_sync(0xffffffffu, c1);
-        c2 = __reduce_add_sync(0xffffffffu, c2);
-        if (lane == 0) {
-            sh.bcnt[buf][d1 - 1] = d1 < nd ? c1 : 0;
-            sh.bcnt[buf][d2 - 1] = d2 < nd ? c2 : 0;
-        }
-        __syncthreads();
-        uint32_t dig = 0;  // digit 0 always holds: count(>= T) >= k
-#pragma unroll
-        for (int d = 1; d < 16; ++d)
-            if (sh.bcnt[buf][d - 1] >= k) dig = d;  // counts fall with d; past nd they are 0
-        T |= dig << sft;
-        buf ^= 1;  // a warp rewrites this buffer only after the next barrier
-        bit = sft - 1;
-    }
-    int gt = 0;
-#pragma unroll
-    for (int c = 0; c < NK; ++c) gt += 32 * c + lane < n && v[c] > T ? 1 : 0;
-    gt = __reduce_add_sync(0xffffffffu, gt);
-    *T_out = T;
-    *ties_out = k - gt;
-}
-
 template <int D>
 __global__ void __launch_bounds__(FinishCfg<D>::NT, FinishCfg<D>::MIN_BLOCKS)
     finish_kernel(FinishParams p) {
@@ -727,11 +653,7 @@ __global__ void __launch_bounds__(FinishCfg<D>::NT, FinishCfg<D>::MIN_BLOCKS)
                         __syncthreads();
                         uint32_t T;
                         int ties;
-                        if (total <= 32 * kBisectKeys)
-                            cta_kth_bisect<NT, kBisectKeys>(&merged[0].key, 4, total, nsel, sh,
-                                                            &T, &ties);
-                        else
-                            cta_kth<NT>(&merged[0].key, 4, total, nsel, sh, &T, &ties);
+                        cta_kth<NT>(&merged[0].key, 4, total, nsel, sh, &T, &ties);
                         // the selected list: keys > T and the first `ties` keys == T,
                         // in index order (over the keys + phys area)
                         const int mspan = ((total + NW - 1) / NW + 31) / 32 * 32;
