@@ -623,7 +623,7 @@ def run_ours(args, rank, world, local):
         del g8, W8
         torch.cuda.empty_cache()
         # the same step with the top-delta selection (the top d pages plus every
-        # page within delta of the best, at most cap), through its four kernels
+        # page within delta of the best, at most cap): the same two kernels
         W9 = Workload("decode256k")
         td, tdelta, tcap = 128, 40.0, 512
         sel9 = torch.full((W9.q.shape[0], W9.wl.hkv, tcap), -1, dtype=torch.int32, device="cuda")
