@@ -11,7 +11,7 @@
 // tiles through a private shared-memory ring (two 8 KB tiles at D=128)
 // filled by asynchronous copies (score_run in slc_score_impl.cuh).  Three
 // 4-warp CTAs per SM keep 24 tiles (192 KB) in flight.  The sparse decode
-// kernel (slc_decode.cu) scores with the same code.
+// kernel (slc_stream.cu) scores with the same code.
 #include "slc_score_impl.cuh"
 
 namespace slc {
