@@ -10,8 +10,8 @@
 // (persistent) grid takes a contiguous range of them.  Each warp streams its
 // tiles through a private shared-memory ring (two 8 KB tiles at D=128)
 // filled by asynchronous copies (score_run in slc_score_impl.cuh).  Three
-// 4-warp CTAs per SM keep 24 tiles (192 KB) in flight.  The sparse decode
-// kernel (slc_stream.cu) scores with the same code.
+// 4-warp CTAs per SM keep 24 tiles (192 KB) in flight.  The streaming kernel
+// of the sparse decode (slc_stream.cu) scores with the same code.
 #include "slc_score_impl.cuh"
 
 namespace slc {
