@@ -49,7 +49,12 @@
  * NULL = the legacy default stream) and launches nothing when it returns an
  * error.  Arguments that live on the device (block-table entries, lengths,
  * positions) are range-checked by the kernels: a bad entry is skipped and
- * flagged in the device status word instead of being dereferenced.
+ * flagged in the device status word instead of being dereferenced.  Kernels
+ * are launched with programmatic dependent launch (a kernel may start while
+ * the previous one on the stream finishes; it waits before reading that
+ * kernel's results); the launches that scan the page metadata also carry an
+ * L2 access-policy window marking the metadata evict-first for that launch
+ * only (no device setting changes).
  *
  * Devices.  Calls run on the device current on the calling thread.  Each
  * kernel's shared-memory limit, occupancy and cluster capacity are looked
