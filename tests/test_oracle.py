@@ -160,6 +160,28 @@ def test_score_nonnegative_query_uses_kmax():
         np.testing.assert_allclose(s[0, h, :10], want, rtol=1e-13)
 
 
+def test_score_equals_the_sign_split_form():
+    """For a <= b, max(q*a, q*b) is q*b when q >= 0 and q*a otherwise, so the
+    group score is also sum_d Qneg_d * kmin_d + Qpos_d * kmax_d with Qpos_d =
+    sum_h max(q_hd, 0), Qneg_d = sum_h min(q_hd, 0) (the form the GPU scoring
+    evaluates).  Mixed-sign queries and bounds, zeros, group sizes 1 to 8."""
+    for hq, hkv, seed in [(8, 8, 21), (8, 2, 22), (12, 4, 23), (8, 1, 24)]:
+        x = _small_cache(2, hq, hkv, 64, [700, 513], seed=seed)
+        x.q[0, 0, :8] = 0.0
+        kmin, kmax = oracle.page_bounds(x.k_cache, x.block_table, x.seq_lens)
+        s = oracle.page_scores(x.q, kmin, kmax, x.seq_lens, prefix=16, window=64)
+        q = x.q.double().numpy()
+        G = hq // hkv
+        for b, L in enumerate(x.seq_lens.tolist()):
+            n, npre, ws = oracle.page_ranges(L, 16, 64)
+            for h in range(hkv):
+                qg = q[b, h * G:(h + 1) * G]
+                qpos = np.maximum(qg, 0.0).sum(axis=0)
+                qneg = np.minimum(qg, 0.0).sum(axis=0)
+                want = kmin[b, h, npre:ws] @ qneg + kmax[b, h, npre:ws] @ qpos
+                np.testing.assert_allclose(s[b, h, npre:ws], want, rtol=1e-12, atol=1e-12)
+
+
 # ---------------------------------------------------------------- selection
 
 def _brute_force_select(vals, pages, k):
