@@ -1,6 +1,7 @@
 """Host logic of the multi-layer decode step (CPU only): the Full/Shared
 assignment of cross-layer reuse and the packed input layout that lets a
 caller move a step's inputs with one copy."""
+import pytest
 import torch
 
 from sparse_long_context_max_b200 import plan as P
@@ -54,3 +55,20 @@ def test_packed_views_round_trip_through_one_copy():
     dst.copy_(src)
     for name, t in vd.items():
         assert torch.equal(t, want[name]), name
+
+
+class _CacheShape:
+    """Stands in for a PagedCache: DecodeStep reads only its shape before
+    it checks the plan."""
+    num_kv_heads, head_dim = 2, 128
+
+
+def test_decode_step_rejects_a_bad_plan():
+    bt = torch.zeros((2, 8), dtype=torch.int32)
+    caches = [_CacheShape(), _CacheShape()]
+    with pytest.raises(ValueError):  # a Shared layer needs a Full layer before it
+        P.DecodeStep(caches, bt, [P.LayerSpec(256, 16, shared=True), P.LayerSpec(256, 16)],
+                     prefix=16, num_q_heads=8)
+    with pytest.raises(ValueError):  # one cache per layer
+        P.DecodeStep(caches[:1], bt, [P.LayerSpec(256, 16), P.LayerSpec(256, 16)],
+                     prefix=16, num_q_heads=8)
